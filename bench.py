@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Throughput of the MoE routing -> layout -> FP8 dispatch -> combine path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3]
+                    [--impl ours|reference] [--graph]
+
+One step = route + dispatch layout + dispatch + combine over one batch of the
+named workload (default: DeepSeek-V3 prefill shape, T=8192 tokens, H=7168,
+256 experts in 8 groups, top-4 groups, top-8, FP8 1x128 dispatch, BF16
+combine).  Inputs are synthetic and seeded; the expert outputs fed to the
+combine are a device-resident bf16 N(0,1) buffer standing in for the expert
+GEMM, which is not part of this path.
+
+``value`` = tokens of all ranks / (max over ranks of the device time of K
+steps).  Multi-GPU runs are independent replicas (one batch per GPU, no data
+exchange between GPUs; "scaling": "weak").  ``--impl reference`` times the CPU
+oracle on the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gen import CONFIGS, Workload, device_normal_bf16  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of peak) at T=8192,H=7168,top-8"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic_bytes(cfg):
+    """Bytes each kernel must move per step (no re-reads), by kernel."""
+    T, H, k, E, R = cfg.T, cfg.H, cfg.topk, cfg.E, cfg.R
+    S = H // 128
+    disp = T * 2 * H + T * k * (H + 4 * S if cfg.fp8 else 2 * H) + T * k * 4
+    comb = T * k * 2 * H + T * 2 * H + T * k * 8
+    route = T * E * 4 + E * 4 + T * k * 8
+    layout = T * k * 4 * 3 + T * R + T * k * 4  # ids read twice, slot + src written
+    return dict(route=route, layout=layout, dispatch=disp, combine=comb)
+
+
+def peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML (read-only)."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        self.window = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id \
+                if hasattr(torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
+            if bus:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+        self.period = period_s
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(inside) < 3:
+            inside = self.samples
+            window = "whole run (timed region shorter than the sampling period)"
+        names = {
+            0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting",
+        }
+        seen = 0
+        for s in inside:
+            seen |= s[2]
+        reasons = [n for b, n in names.items() if seen & b]
+        return {"sm_mhz": statistics.median([s[1] for s in inside]) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "window": window}
+
+
+def cpu_oracle_sample(cfg, wl, y_host_rows, n_tok):
+    """Oracle route+layout+dispatch+combine on the first n_tok tokens."""
+    import oracle
+    sub = cfg.scaled(n_tok)
+    lg = wl.logits[:n_tok].numpy()
+    x = wl.x_rows(0, n_tok)
+    t0 = time.perf_counter()
+    idx, w, _ = oracle.route(lg, wl.bias, sub.n_group, sub.topk_group, sub.topk,
+                             sub.routed_scale, sub.renorm)
+    po = None if wl.phys_of is None else wl.phys_of.numpy()
+    nr = None if wl.n_rep is None else wl.n_rep.numpy()
+    lay = oracle.layout(idx, sub.E, sub.n_phys, sub.R, po, nr)
+    oracle.dispatch(x, lay["slot"], sub.fp8)
+    oracle.combine(y_host_rows, lay["slot"], w)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, cfg):
+    """The oracle on the host cores: each step is a bounded token sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    n_tok = min(cfg.T, args.ref_tokens)
+    wl = Workload(cfg)
+    g = torch.Generator().manual_seed(7)
+    y = torch.randn((n_tok * cfg.topk, cfg.H), generator=g).to(torch.bfloat16)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(cfg, wl, y, n_tok)
+    times = [cpu_oracle_sample(cfg, wl, y, n_tok) for _ in range(args.steps)]
+    tot = sum(times)
+    value = n_tok * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "topk": cfg.topk,
+                   "sample_tokens": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {n_tok} of {cfg.T} tokens per step, single thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="v3", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    ap.add_argument("--num-sms", type=int, default=0)
+    ap.add_argument("--ref-tokens", type=int, default=512,
+                    help="tokens per oracle step (--impl reference and cpu_baseline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from combine_ep_route_02_b200 import EpPath
+
+    wl = Workload(cfg, seed=rank)
+    x_h = wl.x.pin_memory()
+    lg_h = wl.logits.pin_memory()
+    b_h = wl.bias.pin_memory()
+    x, lg, bias = x_h.cuda(), lg_h.cuda(), b_h.cuda()
+    y = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=rank)
+    path = EpPath(cfg.T, cfg.H, cfg.E, cfg.n_group, cfg.topk_group, cfg.topk, cfg.routed_scale,
+                  cfg.renorm, cfg.R, cfg.fp8, phys_of=wl.phys_of, n_rep=wl.n_rep,
+                  num_sms=args.num_sms)
+    stream = torch.cuda.current_stream()
+    ab = algorithmic_bytes(cfg)
+    step_bytes = sum(ab.values())
+    flush = step_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda") if flush else None
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def step():
+        path.step(x, lg, bias, y)
+
+    graph = None
+    if args.graph:
+        s = torch.cuda.Stream()
+        s.wait_stream(stream)
+        with torch.cuda.stream(s):
+            step()
+        stream.wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    path.check_status()
+
+    # kernel-level events (combine = dominant kernel) are recorded inside the
+    # timed region on the launching stream; they need eager launches
+    kev = graph is None
+    K = args.steps
+    c0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
+    c1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
+    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
+    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
+    s0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    s1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(K):
+        if flush:
+            flush_buf.fill_(i & 0xFF)  # evict the previous step's data from L2
+        s0[i].record(stream)
+        if kev:
+            path.route(lg, bias)
+            path.layout()
+            d0[i].record(stream)
+            path.dispatch(x)
+            d1[i].record(stream)
+            c0[i].record(stream)
+            path.combine(y)
+            c1[i].record(stream)
+        else:
+            run_step()
+        s1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.perf_counter()
+    sampler.stop()
+    path.check_status()
+
+    step_ms = [a.elapsed_time(b) for a, b in zip(s0, s1)]
+    tot_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([tot_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    value = cfg.T * world * K / (tot_ms * 1e-3)
+
+    peak, peak_kind = peak_hbm()
+    roofline = None
+    extra = {}
+    if kev:
+        comb_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(c0, c1))
+        disp_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(d0, d1))
+        comb_gbs = ab["combine"] / (comb_ms * 1e-3) / 1e9
+        disp_gbs = ab["dispatch"] / (disp_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "combine_kernel", "achieved": comb_gbs,
+                    "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
+                    "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy)"
+                    if peak_kind == "measured" else "fallback 6650 GB/s",
+                    "traffic": None}
+        dc_ms = comb_ms + disp_ms
+        extra = {
+            "dispatch_us": disp_ms * 1e3, "combine_us": comb_ms * 1e3,
+            "dispatch_gbs": disp_gbs, "combine_gbs": comb_gbs,
+            "dispatch_combine_tokens_per_s": cfg.T * world / (dc_ms * 1e-3),
+            "dispatch_combine_gbs": (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3) / 1e9,
+            "dispatch_combine_frac_of_peak": (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3)
+            / 1e9 / peak,
+            "step_gbs": step_bytes / (tot_ms / K * 1e-3) / 1e9,
+        }
+
+    # end to end through the public API: host inputs in, host result out
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+        for _ in range(max(3, args.warmup // 2)):
+            x.copy_(x_h, non_blocking=True)
+            lg.copy_(lg_h, non_blocking=True)
+            bias.copy_(b_h, non_blocking=True)
+            run_step()
+            out_h.copy_(path.out, non_blocking=True)
+        Ke = max(3, min(K, 50))
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            x.copy_(x_h, non_blocking=True)
+            lg.copy_(lg_h, non_blocking=True)
+            bias.copy_(b_h, non_blocking=True)
+            run_step()
+            out_h.copy_(path.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ems], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = x_h.numel() * 2 + lg_h.numel() * 4 + b_h.numel() * 4
+        e2e = {"value": cfg.T * world * Ke / (ems * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_h.numel() * 2,
+               "steps": Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok = min(cfg.T, args.ref_tokens)
+        yh = y[: n_tok * cfg.topk].cpu()
+        secs = cpu_oracle_sample(cfg, wl, yh, n_tok)
+        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {n_tok} of {cfg.T} tokens of the same workload, one pass of "
+                         f"route+layout+dispatch+combine, single thread ({secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": tot_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 accumulate",
+            "data": "synthetic (seeded SplitMix64 / Box-Muller inputs; expert outputs bf16 N(0,1))",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                       "P": cfg.n_phys, "R": cfg.R, "n_group": cfg.n_group,
+                       "topk_group": cfg.topk_group, "topk": cfg.topk, "fp8": cfg.fp8,
+                       "routed_scale": cfg.routed_scale, "cuda_graph": graph is not None,
+                       "l2": ("flushed before each step (256 MiB write, outside step events)"
+                              if flush else
+                              f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB moved per step)"),
+                       "parallelism": f"replicas x{world}"},
+            "gpu_launches": path.kernels_per_step() * K,
+            "roofline": roofline,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": sampler.summary(t_wall0, t_wall1),
+            "wall_s_timed": t_wall1 - t_wall0,
+            **extra,
+        }
+        print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

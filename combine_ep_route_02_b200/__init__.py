@@ -1,0 +1,28 @@
+"""B200 (sm_100a) MoE expert-parallel routing, dispatch layout, FP8 dispatch
+and weighted combine on one GPU.
+
+The compute lives in ``lib/libep_b200.so`` (C ABI in ``include/ep.h``); this
+package is its ctypes binding plus ``EpPath``, which owns the device buffers
+for one shape.  Importing the package does not load the library; the first
+call does, and raises if it has not been built.
+"""
+
+from ._binding import (  # noqa: F401
+    EP_DEV_BAD_EXPERT,
+    EP_DEV_BAD_REPLICA,
+    EP_ERR_CUDA,
+    EP_ERR_DEVICE,
+    EP_ERR_INVALID,
+    EP_ERR_UNSUPPORTED,
+    EP_OK,
+    EXPORTS,
+    EpError,
+    RouteCfg,
+    ep_combine,
+    ep_dispatch,
+    ep_dispatch_layout,
+    ep_route,
+    ep_workspace_size,
+    lib,
+)
+from .path import EpPath  # noqa: F401

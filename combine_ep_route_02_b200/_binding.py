@@ -1,0 +1,120 @@
+"""ctypes binding of libep_b200.so: the C-ABI calls under the same names.
+
+Argument marshalling only: tensors become device pointers, the current torch
+stream becomes the stream handle, ep_status codes become exceptions.  Every
+step of the path runs in the library's CUDA kernels; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+_lib = None
+
+EP_OK = 0
+EP_ERR_INVALID = 1
+EP_ERR_UNSUPPORTED = 2
+EP_ERR_CUDA = 3
+EP_ERR_DEVICE = 4
+EP_DEV_BAD_EXPERT = 1
+EP_DEV_BAD_REPLICA = 2
+
+# every symbol declared in include/ep.h
+EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
+           "ep_combine", "ep_status_string")
+
+
+class EpError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        msg = lib().ep_status_string(status).decode()
+        super().__init__(f"{fn}: {msg}")
+
+
+class RouteCfg(ctypes.Structure):
+    _fields_ = [("num_experts", ctypes.c_int), ("n_group", ctypes.c_int),
+                ("topk_group", ctypes.c_int), ("topk", ctypes.c_int),
+                ("routed_scale", ctypes.c_float), ("renorm", ctypes.c_int)]
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise ImportError(
+                f"libep_b200.so not found at {LIB}; build it with "
+                "`python -m combine_ep_route_02_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB)
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.ep_workspace_size.argtypes = [I, I, I, I]
+        L.ep_workspace_size.restype = Z
+        L.ep_route.argtypes = [P, P, I, RouteCfg, P, P, P]
+        L.ep_route.restype = I
+        L.ep_dispatch_layout.argtypes = [P, I, I, I, I, I, P, P, I,
+                                         P, P, P, P, P, P, P, P, P, P, P]
+        L.ep_dispatch_layout.restype = I
+        L.ep_dispatch.argtypes = [P, I, I, I, P, I, P, P, I, P]
+        L.ep_dispatch.restype = I
+        L.ep_combine.argtypes = [P, P, P, I, I, I, P, I, P]
+        L.ep_combine.restype = I
+        L.ep_status_string.argtypes = [I]
+        L.ep_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, st):
+    if st != EP_OK:
+        raise EpError(fn, st)
+
+
+def ep_workspace_size(T: int, k: int, P: int, R: int) -> int:
+    return int(lib().ep_workspace_size(T, k, P, R))
+
+
+def ep_route(logits, bias, T, cfg: RouteCfg, topk_idx, topk_w, stream=None):
+    _check("ep_route", lib().ep_route(_ptr(logits), _ptr(bias), T, cfg, _ptr(topk_idx),
+                                      _ptr(topk_w), _stream(stream)))
+
+
+def ep_dispatch_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
+                       expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
+                       workspace, dev_status, stream=None):
+    _check("ep_dispatch_layout", lib().ep_dispatch_layout(
+        _ptr(topk_idx), T, k, E, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
+        _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank), _ptr(rank_off), _ptr(tok_rank),
+        _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace), _ptr(dev_status),
+        _stream(stream)))
+
+
+def ep_dispatch(x, T, H, k, slot, fp8, recv_x, recv_scale, num_sms=0, stream=None):
+    _check("ep_dispatch", lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot), int(bool(fp8)),
+                                            _ptr(recv_x), _ptr(recv_scale), num_sms,
+                                            _stream(stream)))
+
+
+def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, stream=None):
+    _check("ep_combine", lib().ep_combine(_ptr(y), _ptr(slot), _ptr(topk_w), T, H, k,
+                                          _ptr(out), num_sms, _stream(stream)))

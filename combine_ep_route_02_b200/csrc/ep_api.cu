@@ -1,0 +1,148 @@
+// C-ABI entry points of libep_b200: host-side argument checks, launch
+// configuration, and the mapping of CUDA errors to ep_status.
+#include "../../include/ep.h"
+#include "ep_internal.h"
+
+namespace ep {
+
+int device_sm_count()
+{
+    static volatile int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+ep_status from_cuda(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+// grid of a streaming kernel: num_sms SMs (0 = all) x resident blocks per SM
+int streaming_grid(int num_sms, int blocks_per_sm)
+{
+    const int sms = device_sm_count();
+    const int use = (num_sms <= 0 || num_sms > sms) ? sms : num_sms;
+    return use * blocks_per_sm;
+}
+
+int cached_blocks_per_sm(int which)
+{
+    // which: 0 = dispatch bf16, 1 = dispatch fp8, 2 = combine
+    static volatile int cache[64][3] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && cache[dev][which] > 0) return cache[dev][which];
+    const int n = which == 2 ? combine_blocks_per_sm() : dispatch_blocks_per_sm(which);
+    if (dev < 64) cache[dev][which] = n;
+    return n;
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" {
+
+const char *ep_status_string(ep_status s)
+{
+    switch (s) {
+    case EP_OK: return "EP_OK";
+    case EP_ERR_INVALID: return "EP_ERR_INVALID: invalid argument";
+    case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED: size above a library limit";
+    case EP_ERR_CUDA: return "EP_ERR_CUDA: CUDA launch or API error";
+    case EP_ERR_DEVICE: return "EP_ERR_DEVICE: bad data reported by the device";
+    }
+    return "unknown ep_status";
+}
+
+size_t ep_workspace_size(int T, int k, int P, int R)
+{
+    if (T < 0 || k < 1 || P < 1 || R < 1) return 0;
+    const size_t NT = (size_t)layout_tiles(T > 0 ? T : 1);
+    return align256(NT * (size_t)P * sizeof(int32_t)) + align256(NT * (size_t)R * sizeof(int32_t));
+}
+
+ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                   int32_t *topk_idx, float *topk_w, ep_stream_t stream)
+{
+    const int E = cfg.num_experts, G = cfg.n_group, Kg = cfg.topk_group, k = cfg.topk;
+    if (T < 0 || E < 1 || G < 1 || Kg < 1 || k < 1) return EP_ERR_INVALID;
+    if (E % G != 0 || Kg > G || (G > 1 && E / G < 2)) return EP_ERR_INVALID;
+    if ((long long)k > (long long)(E / G) * Kg) return EP_ERR_INVALID;
+    if (E > MAX_EXPERTS || G > MAX_GROUPS || k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * E >= (1LL << 31) || (long long)T * k >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!logits || !topk_idx || !topk_w)) return EP_ERR_INVALID;
+    if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return EP_ERR_INVALID;
+    RouteArgs a{logits, bias, T, E, G, Kg, k, cfg.routed_scale, cfg.renorm != 0, topk_idx, topk_w};
+    return from_cuda(launch_route(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                             const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
+                             int32_t *slot, int32_t *src, void *workspace,
+                             int32_t *dev_status, ep_stream_t stream)
+{
+    if (T < 0 || k < 1 || E < 1 || P < 1 || R < 1) return EP_ERR_INVALID;
+    if (P % R != 0) return EP_ERR_INVALID;
+    if ((phys_of == nullptr) != (n_rep == nullptr)) return EP_ERR_INVALID;
+    if (phys_of == nullptr && P != E) return EP_ERR_INVALID;
+    if (phys_of != nullptr && (P < E || max_rep < 1)) return EP_ERR_INVALID;
+    if (k > MAX_TOPK || P > MAX_PHYS) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31) || (long long)T * R >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if (!cnt_expert || !expert_off || !rows_rank || !rank_off || !tok_rank) return EP_ERR_INVALID;
+    if (T > 0 && (!topk_idx || !in_rank || !slot || !src || !workspace)) return EP_ERR_INVALID;
+    if (!aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(slot, 4) || !aligned(src, 4) ||
+        !aligned(dev_status, 4))
+        return EP_ERR_INVALID;
+    const int NT = layout_tiles(T);
+    int32_t *ws = static_cast<int32_t *>(workspace);
+    LayoutArgs a{topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
+                 cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
+                 ws, ws + align256((size_t)NT * P * sizeof(int32_t)) / sizeof(int32_t),
+                 dev_status};
+    return from_cuda(launch_layout(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
+                      void *recv_x, float *recv_scale, int num_sms, ep_stream_t stream)
+{
+    if (T < 0 || H < 1 || k < 1) return EP_ERR_INVALID;
+    if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_INVALID;
+    if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!x_bf16 || !slot || !recv_x || (fp8 && !recv_scale))) return EP_ERR_INVALID;
+    if (!aligned(x_bf16, 16) || !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(slot, 4))
+        return EP_ERR_INVALID;
+    DispatchArgs a{x_bf16, T, H, k, slot, fp8 != 0, recv_x, recv_scale,
+                   streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0))};
+    return from_cuda(launch_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T, int H,
+                     int k, void *out_bf16, int num_sms, ep_stream_t stream)
+{
+    if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
+    if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!y_bf16 || !slot || !topk_w || !out_bf16)) return EP_ERR_INVALID;
+    if (!aligned(y_bf16, 16) || !aligned(out_bf16, 16) || !aligned(slot, 4) || !aligned(topk_w, 4))
+        return EP_ERR_INVALID;
+    CombineArgs a{y_bf16, slot, topk_w, T, H, k, out_bf16,
+                  streaming_grid(num_sms, cached_blocks_per_sm(2))};
+    return from_cuda(launch_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -10,6 +10,7 @@ from .inputs import (  # noqa: F401
     CONFIGS,
     Workload,
     WorkloadConfig,
+    device_normal_bf16,
     expert_permutation,
     normals,
     redundant_expert_map,

@@ -211,8 +211,8 @@ class Workload:
     def __init__(self, cfg: WorkloadConfig, seed: int = 0):
         self.cfg = cfg
         self.seed = seed
-        T, H, E = cfg.T, cfg.H, cfg.E
-        self.x = _to_bf16(normals(stream_key(seed, STREAM_X), 0, T * H)).view(T, H)
+        T, E = cfg.T, cfg.E
+        self._x = None
         self.logits = torch.from_numpy(
             normals(stream_key(seed, STREAM_LOGITS), 0, T * E).astype(np.float32)
         ).view(T, E)
@@ -234,6 +234,17 @@ class Workload:
             self.phys_of, self.n_rep = (torch.from_numpy(a) for a in redundant_expert_map(
                 pi, cfg.R, cfg.P // cfg.R, cfg.n_hot, cfg.zipf_s))
 
+    @property
+    def x(self) -> torch.Tensor:
+        if self._x is None:
+            T, H = self.cfg.T, self.cfg.H
+            self._x = _to_bf16(normals(stream_key(self.seed, STREAM_X), 0, T * H)).view(T, H)
+        return self._x
+
+    def x_rows(self, first: int, n: int) -> torch.Tensor:
+        H = self.cfg.H
+        return _to_bf16(normals(stream_key(self.seed, STREAM_X), first * H, n * H)).view(n, H)
+
     def y_rows(self, first: int, n: int) -> torch.Tensor:
         H = self.cfg.H
         v = normals(stream_key(self.seed, STREAM_Y), first * H, n * H)
@@ -241,3 +252,19 @@ class Workload:
 
     def y(self) -> torch.Tensor:
         return self.y_rows(0, self.cfg.T * self.cfg.topk)
+
+
+def device_normal_bf16(rows: int, cols: int, seed: int, device="cuda") -> torch.Tensor:
+    """bf16 N(0,1) [rows, cols] drawn on the device by torch's seeded Philox
+    generator: a large stand-in input (e.g. expert outputs) that would take
+    too long to draw on the host.  Both the GPU path and the oracle read the
+    same bytes (the oracle after a copy to the host)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(0x5EED0000 + seed)
+    out = torch.empty((rows, cols), device=device, dtype=torch.bfloat16)
+    step = max(1, (1 << 26) // max(cols, 1))
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        out[r0:r1] = torch.randn((r1 - r0, cols), generator=g, device=device,
+                                 dtype=torch.float32).to(torch.bfloat16)
+    return out

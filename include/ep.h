@@ -1,0 +1,194 @@
+/*
+ * ep.h -- C ABI of the B200 (sm_100a) MoE expert-parallel routing, dispatch
+ * layout, FP8 dispatch and combine library (libep_b200.so).
+ *
+ * The operations are the four steps around the experts of a MoE layer:
+ *
+ *   ep_route            gate logits -> top-k expert ids and weights
+ *   ep_dispatch_layout  top-k ids   -> per-expert / per-rank counts, prefix
+ *                                      sums, receive-row slots
+ *   ep_dispatch         tokens      -> rank-major, expert-contiguous receive
+ *                                      rows (BF16 copies, or e4m3 + 1x128
+ *                                      scales)
+ *   ep_combine          expert rows -> top-k weighted sum per token (BF16)
+ *
+ * Sources (page title, then section):
+ *  - Perplexity, "Lower latency and higher throughput with multi-node
+ *    DeepSeek deployment": section "Expert Parallelism" (256 routed experts,
+ *    8 per token, weighted sum; dispatch and combine are the two all-to-alls
+ *    around the experts), section "Quantization" (1x128 activation scales,
+ *    M x ceil_div(K,128) of them, amax over 128-element sub-blocks), section
+ *    "MoE Router" (Mixtral top-k is DeepSeek group routing with one group;
+ *    dense dispatch/combine plans need per-expert aggregates), section
+ *    "CUDA Graph" (kernels read the routing counts instead of sizing work from
+ *    buffer capacities, so they can be captured).
+ *  - DeepEP V2 summary (news.hada.io, "DeepSeek merilis library open source
+ *    DeepEP"), section on the ElasticBuffer interface (buffer size hint,
+ *    num_sms override) and section "Usage for training, prefill and
+ *    decoding" (the dispatch handle carries num_recv_tokens_per_expert_list
+ *    for the GEMM; combine reduces expert outputs back to the source; a
+ *    cached handle skips the layout in decoding).
+ *  - DeepSeek Open Infra day-4 summary, EPLB section (group-limited routing;
+ *    redundant experts replicated and placed across GPUs).
+ *
+ * On one GPU the expert-parallel ranks are logical: rank r owns physical
+ * experts [r*P/R, (r+1)*P/R) and its receive rows are the contiguous range
+ * [rank_off[r], rank_off[r+1]) of one buffer.
+ *
+ * Conventions for every entry point
+ *  - Memory: every array pointer is DEVICE memory allocated and freed by the
+ *    caller.  The library allocates nothing, frees nothing, keeps no state
+ *    between calls and never synchronises the host.  All work is enqueued on
+ *    `stream` (NULL = the legacy default stream).
+ *  - Layout: row-major, densely packed.  Index arrays are int32.
+ *  - Errors: argument checks happen on the host before anything is enqueued
+ *    and return EP_ERR_INVALID (bad shape / value / alignment) or
+ *    EP_ERR_UNSUPPORTED (valid but beyond this build's limits).  A launch
+ *    failure returns EP_ERR_CUDA.  Bad data found on the device (an expert id
+ *    outside [0,E), an invalid replica map entry) never traps: it sets bits
+ *    in the caller's *dev_status and the offending pair gets slot -1.
+ *  - Empty input (T == 0) is valid and produces empty / zero outputs.
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID = 1,     /* bad argument: shape, value, alignment, NULL */
+    EP_ERR_UNSUPPORTED = 2, /* valid but above a limit of this library */
+    EP_ERR_CUDA = 3,        /* a CUDA launch or API call failed */
+    EP_ERR_DEVICE = 4       /* reserved for callers mapping *dev_status */
+} ep_status;
+
+/* Bits written to *dev_status by ep_dispatch_layout. */
+#define EP_DEV_BAD_EXPERT 1  /* a topk_idx entry outside [0, E) */
+#define EP_DEV_BAD_REPLICA 2 /* n_rep[e] outside [1, max_rep] or phys id outside [0, P) */
+
+/* Same object as cudaStream_t; no CUDA header is needed to use this API. */
+typedef struct CUstream_st *ep_stream_t;
+
+/* Routing configuration.
+ *   num_experts   E, 1..1024
+ *   n_group       G: experts form G runs of E/G consecutive ids; 1..32,
+ *                 E % G == 0, and E/G >= 2 when G > 1
+ *   topk_group    groups kept per token, 1..G
+ *   topk          k experts per token, 1..32, k <= (E/G) * topk_group
+ *   routed_scale  multiplies every weight (2.5 for DeepSeek-V3)
+ *   renorm        nonzero: weights are divided by their sum before scaling */
+typedef struct {
+    int num_experts;
+    int n_group;
+    int topk_group;
+    int topk;
+    float routed_scale;
+    int renorm;
+} ep_route_cfg;
+
+/*
+ * Bytes of device scratch that ep_dispatch_layout needs for T tokens, top-k,
+ * P physical experts and R logical ranks (the counterpart of DeepEP's buffer
+ * size hint).  Returns 0 for invalid sizes.  The scratch need not be zeroed.
+ */
+size_t ep_workspace_size(int T, int k, int P, int R);
+
+/*
+ * Sigmoid-gated, group-limited top-k routing (DeepSeek-V3 style; EPLB
+ * section of the DeepSeek Open Infra summary, MoE Router section of the
+ * Perplexity blog).
+ *
+ *   logits    fp32 [T, E]
+ *   bias      fp32 [E] selection bias, or NULL for none
+ *   topk_idx  int32 [T, k] (out)  chosen expert ids in selection order
+ *   topk_w    fp32  [T, k] (out)  weights
+ *
+ * Per token: s_e = fp32(1/(1+exp(-x_e))) evaluated in fp64; key_e = s_e + b_e
+ * (fp32).  With G > 1 a group scores the fp32 sum of its two largest keys and
+ * only the topk_group best groups stay eligible.  The k largest keys among the
+ * eligible experts are chosen, ties to the lower index (groups: ties to the
+ * lower group id).  w_j = s_{e_j}; with renorm, w_j /= sum_j w_j (fp32, in j
+ * order; skipped when the sum is 0); then w_j *= routed_scale.  Every fp32
+ * operation rounds once to nearest even.
+ */
+ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                   int32_t *topk_idx, float *topk_w, ep_stream_t stream);
+
+/*
+ * Dispatch layout: counts, prefix sums and deterministic slots (the
+ * "handle" of DeepEP V2; num_recv_tokens_per_expert_list = cnt_expert).
+ *
+ *   topk_idx   int32 [T, k] logical expert ids in [0, E)
+ *   E, P, R    logical experts, physical experts, logical ranks; P % R == 0;
+ *              P == E unless a replica map is given (then P >= E)
+ *   phys_of    int32 [E, max_rep] or NULL: physical ids of each expert's
+ *              replicas; token t uses replica phys_of[e][t % n_rep[e]]
+ *   n_rep      int32 [E] or NULL (together with phys_of)
+ *   outputs    cnt_expert [P]     rows per physical expert
+ *              expert_off [P+1]   exclusive prefix sum of cnt_expert
+ *              rows_rank  [R]     rows per rank (sum of its experts' counts)
+ *              rank_off   [R+1]   exclusive prefix sum of rows_rank
+ *              tok_rank   [R]     tokens with at least one expert on the rank
+ *              in_rank    uint8 [T, R]  1 if token t sends to rank r
+ *              slot       [T, k]  receive row of pair (t, j); -1 if invalid
+ *              src        [T*k]   inverse of slot: src[slot[t,j]] = t*k + j
+ *   workspace  ep_workspace_size(T, k, P, R) bytes, 256-byte aligned
+ *   dev_status int32 [1] or NULL; zeroed by this call, then EP_DEV_* bits
+ *
+ * Receive rows are ordered by physical expert, and within an expert by
+ * (t, j); there is no padding, so valid pairs fill rows [0, expert_off[P]).
+ * Rank r's rows are [rank_off[r], rank_off[r+1]).  The result does not
+ * depend on scheduling (no global atomics decide an order).
+ */
+ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                             const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
+                             int32_t *slot, int32_t *src, void *workspace,
+                             int32_t *dev_status, ep_stream_t stream);
+
+/*
+ * Dispatch (permute, optionally with fused 1x128 FP8 quantisation).
+ *
+ *   x_bf16      bf16 [T, H], 16-byte aligned; H % 8 == 0 (H % 128 == 0 for fp8)
+ *   slot        int32 [T, k] from ep_dispatch_layout (or a cached copy)
+ *   fp8 == 0:   recv_x is bf16 [T*k, H]; row slot[t,j] = x[t] bit for bit
+ *   fp8 != 0:   recv_x is e4m3fn [T*k, H] and recv_scale fp32 [T*k, H/128];
+ *               per 128-element block b of x[t]: amax = max|x|, scale =
+ *               fp32(amax / 448), q = e4m3_rn_satfinite(fp32(x / scale));
+ *               a block with amax == 0 gets scale 0 and zero bytes
+ *   num_sms     SMs to spread the work over (0 = all), like DeepEP's num_sms
+ *
+ * Slots outside [0, T*k) are skipped (rows they would fill are left as they
+ * were).  recv_x must be 16-byte aligned, recv_scale 4-byte aligned.
+ */
+ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
+                      void *recv_x, float *recv_scale, int num_sms, ep_stream_t stream);
+
+/*
+ * Combine: weighted gather-reduce back to token order.
+ *
+ *   y_bf16    bf16 [T*k, H] expert outputs in receive-row order
+ *   slot      int32 [T, k], topk_w fp32 [T, k]
+ *   out_bf16  bf16 [T, H] (out)
+ *
+ * out[t] = bf16_rne( acc ), acc = fp32 sum over j = 0..k-1 in order of
+ * fp32(w[t,j] * y[slot[t,j]]), each step rounded to nearest even.  Slots
+ * outside [0, T*k) contribute nothing.  y and out 16-byte aligned, H % 8 == 0.
+ */
+ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T,
+                     int H, int k, void *out_bf16, int num_sms, ep_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *ep_status_string(ep_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

@@ -1,0 +1,422 @@
+"""CUDA path (through the C ABI) vs the CPU oracle, element by element.
+
+Routing indices and weights, every layout array, FP8 payload bytes and
+scales, and BF16 dispatch rows must be bit-identical; the BF16 combine must
+lie within |d| <= 1e-3 + 1e-2 |oracle| (and is expected to be identical,
+because the kernel rounds in the oracle's order).  Inputs come from the
+seeded generator; nothing the oracle reads comes from the CUDA path.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen import CONFIGS, Workload, device_normal_bf16
+from tests._common import (LAYOUT_FIELDS, assert_combine_close, gpu_layout_dict, make_path,
+                           oracle_layout, oracle_route, u16, workload)
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny", "ds16b", "v3", "v3_decode", "skew"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from combine_ep_route_02_b200 import build
+    build.build()
+    yield
+    torch.cuda.synchronize()
+
+
+def check_route(cfg, wl, gidx, gw):
+    idx, w, hard = oracle_route(cfg, wl)
+    ok = hard == 0
+    assert np.array_equal(gidx[ok], idx[ok])
+    assert np.array_equal(gw[ok].view(np.uint32), w[ok].view(np.uint32))
+    # tokens holding a sigmoid within 2^-47 of an fp32 midpoint: valid routing
+    for t in np.nonzero(~ok)[0]:
+        assert len(set(gidx[t])) == cfg.topk
+    return int((~ok).sum())
+
+
+# ---------------------------------------------------------------------------
+# routing
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ALL)
+def test_route_full_size(name):
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    path = make_path(cfg, wl)
+    path.route(wl.logits.cuda(), wl.bias.cuda())
+    torch.cuda.synchronize()
+    n_hard = check_route(cfg, wl, path.topk_idx.cpu().numpy(), path.topk_w.cpu().numpy())
+    assert n_hard <= 2
+
+
+ROUTE_SHAPES = [  # E, G, Kg, k
+    (16, 1, 1, 2), (30, 1, 1, 3), (64, 1, 1, 6), (128, 4, 2, 8), (132, 2, 1, 7),
+    (256, 8, 4, 8), (288, 8, 3, 9), (512, 16, 4, 8), (1024, 32, 8, 32), (24, 3, 2, 5),
+    (256, 32, 1, 8), (96, 32, 32, 32),
+]
+
+
+@pytest.mark.parametrize("E,G,Kg,k", ROUTE_SHAPES)
+@pytest.mark.parametrize("kind", ["normal", "grid", "nobias"])
+def test_route_shapes(E, G, Kg, k, kind):
+    rng = np.random.default_rng(E * 7 + G * 3 + k)
+    T = 203
+    if kind == "grid":  # frequent exact ties among keys and group scores
+        logits = rng.choice([-1.0, 0.0, 1.0], size=(T, E)).astype(np.float32)
+    else:
+        logits = rng.normal(0, 1, (T, E)).astype(np.float32)
+    bias = None if kind == "nobias" else rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    for scale, renorm in [(2.5, True), (1.0, False)]:
+        from combine_ep_route_02_b200 import RouteCfg, ep_route
+        cfg = RouteCfg(E, G, Kg, k, scale, int(renorm))
+        lg = torch.from_numpy(logits).cuda()
+        bs = None if bias is None else torch.from_numpy(bias).cuda()
+        gidx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        ep_route(lg, bs, T, cfg, gidx, gw)
+        idx, w, hard = oracle.route(logits, bias, G, Kg, k, scale, renorm)
+        ok = hard == 0
+        gi, gwn = gidx.cpu().numpy(), gw.cpu().numpy()
+        assert np.array_equal(gi[ok], idx[ok])
+        assert np.array_equal(gwn[ok].view(np.uint32), w[ok].view(np.uint32))
+
+
+def test_route_empty_and_single():
+    from combine_ep_route_02_b200 import RouteCfg, ep_route
+    cfg = RouteCfg(256, 8, 4, 8, 2.5, 1)
+    gidx = torch.full((1, 8), -7, dtype=torch.int32, device="cuda")
+    gw = torch.zeros((1, 8), dtype=torch.float32, device="cuda")
+    ep_route(torch.empty((0, 256), device="cuda"), None, 0, cfg, gidx, gw)
+    torch.cuda.synchronize()
+    assert (gidx == -7).all()
+    lg = torch.randn((1, 256), generator=torch.Generator().manual_seed(3))
+    ep_route(lg.cuda(), None, 1, cfg, gidx, gw)
+    idx, w, _ = oracle.route(lg, None, 8, 4, 8, 2.5, True)
+    assert np.array_equal(gidx.cpu().numpy(), idx)
+    assert np.array_equal(gw.cpu().numpy().view(np.uint32), w.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# layout
+# ---------------------------------------------------------------------------
+
+def run_layout(cfg, wl, topk_idx_np):
+    path = make_path(cfg, wl)
+    path.topk_idx.copy_(torch.from_numpy(topk_idx_np))
+    path.layout()
+    torch.cuda.synchronize()
+    return path
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_layout_full_size(name):
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    idx, _, _ = oracle_route(cfg, wl)
+    path = run_layout(cfg, wl, idx)
+    ref = oracle_layout(cfg, wl, idx)
+    got = gpu_layout_dict(path)
+    assert ref["status"] == 0 and int(path.dev_status.item()) == 0
+    for n in LAYOUT_FIELDS:
+        assert np.array_equal(got[n].reshape(ref[n].shape), ref[n]), n
+
+
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 1000, 4097])
+@pytest.mark.parametrize("name", ["ds16b", "skew"])
+def test_layout_ragged(T, name):
+    cfg = CONFIGS[name].scaled(T)
+    wl = Workload(cfg, seed=T)
+    idx, _, _ = oracle_route(cfg, wl)
+    path = run_layout(cfg, wl, idx)
+    ref = oracle_layout(cfg, wl, idx)
+    got = gpu_layout_dict(path)
+    for n in LAYOUT_FIELDS:
+        assert np.array_equal(got[n].reshape(ref[n].shape), ref[n]), n
+
+
+def test_layout_empty():
+    cfg = CONFIGS["v3"].scaled(0)
+    path = make_path(cfg, Workload(cfg))
+    for n in ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank"):
+        getattr(path, n).fill_(-5)
+    path.layout()
+    torch.cuda.synchronize()
+    for n in ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank"):
+        assert (getattr(path, n) == 0).all(), n
+
+
+def test_layout_max_sizes_and_skewed_ids():
+    """P = 4096 physical experts, k = 32, R = 64, heavily skewed expert ids"""
+    from combine_ep_route_02_b200 import ep_dispatch_layout, ep_workspace_size
+    rng = np.random.default_rng(11)
+    T, k, E, R = 700, 32, 4096, 64
+    idx = np.stack([rng.choice(E, k, replace=False, p=None) for _ in range(T)]).astype(np.int32)
+    idx[::3, :8] = np.arange(8)  # many tokens on the same few experts
+    ref = oracle.layout(idx, E, E, R)
+    d = dict(cnt_expert=E, expert_off=E + 1, rows_rank=R, rank_off=R + 1, tok_rank=R,
+             slot=(T, k), src=T * k)
+    g = {n: torch.empty(s, dtype=torch.int32, device="cuda") for n, s in d.items()}
+    in_rank = torch.empty((T, R), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ep_workspace_size(T, k, E, R), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ep_dispatch_layout(torch.from_numpy(idx).cuda(), T, k, E, E, R, None, None, 0,
+                       g["cnt_expert"], g["expert_off"], g["rows_rank"], g["rank_off"],
+                       g["tok_rank"], in_rank, g["slot"], g["src"], ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for n in d:
+        assert np.array_equal(g[n].cpu().numpy().reshape(ref[n].shape), ref[n]), n
+    assert np.array_equal(in_rank.cpu().numpy(), ref["in_rank"])
+
+
+def test_layout_bad_ids_set_status():
+    cfg = CONFIGS["skew"].scaled(300)
+    wl = Workload(cfg)
+    idx, _, _ = oracle_route(cfg, wl)
+    idx[5, 2] = 256        # out of range
+    idx[77, 0] = -3
+    path = run_layout(cfg, wl, idx)
+    ref = oracle_layout(cfg, wl, idx)
+    assert ref["status"] == oracle.BAD_EXPERT
+    assert int(path.dev_status.item()) == ref["status"]
+    got = gpu_layout_dict(path)
+    for n in ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank", "in_rank", "slot"):
+        assert np.array_equal(got[n].reshape(ref[n].shape), ref[n]), n
+    # a broken replica map is reported too, and never read out of bounds
+    n_rep = wl.n_rep.clone()
+    n_rep[int(idx[9, 1])] = 0
+    path2 = make_path(cfg, wl)
+    path2.n_rep.copy_(n_rep)
+    path2.topk_idx.copy_(torch.from_numpy(idx))
+    path2.layout()
+    ref2 = oracle.layout(idx, cfg.E, cfg.n_phys, cfg.R, wl.phys_of.numpy(), n_rep.numpy())
+    assert int(path2.dev_status.item()) == ref2["status"] == oracle.BAD_EXPERT | oracle.BAD_REPLICA
+    assert np.array_equal(path2.slot.cpu().numpy(), ref2["slot"])
+
+
+# ---------------------------------------------------------------------------
+# dispatch
+# ---------------------------------------------------------------------------
+
+def check_dispatch(cfg, x_cpu, slot_np, path):
+    rx, rs = oracle.dispatch(x_cpu, slot_np, cfg.fp8)
+    if cfg.fp8:
+        got = path.recv_x.view(torch.uint8).cpu().numpy()
+        bad = np.nonzero((got != rx).any(axis=1))[0]
+        assert bad.size == 0, (bad[:5], got[bad[0]][:16], rx[bad[0]][:16])
+        gs = path.recv_scale.cpu().numpy()
+        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32))
+    else:
+        assert np.array_equal(u16(path.recv_x), rx)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_dispatch_full_size(name):
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    idx, _, _ = oracle_route(cfg, wl)
+    lay = oracle_layout(cfg, wl, idx)
+    path = make_path(cfg, wl)
+    path.slot.copy_(torch.from_numpy(lay["slot"]))
+    path.dispatch(wl.x.cuda())
+    torch.cuda.synchronize()
+    check_dispatch(cfg, wl.x, lay["slot"], path)
+
+
+def adversarial_rows(H=1024):
+    """blocks that stress the quantiser: zeros, -0, tiny and huge amax,
+    saturation, exact e4m3 ties after scaling, bf16 subnormals"""
+    rng = np.random.default_rng(12)
+    rows = []
+    nb = H // 128
+
+    def row(blocks):
+        return np.concatenate(blocks).astype(np.float32)
+
+    z = np.zeros(128, np.float32)
+    rows.append(row([z] * nb))
+    rows.append(row([-z] * nb))
+    rows.append(row([np.full(128, 3.0, np.float32)] * nb))                     # all == amax
+    ties = np.array([448.0] + [1.0625, 1.1875, -2.125, 0.0029296875, 0.0009765625] * 25 +
+                    [0.5, 0.25], np.float32)                                  # scale 1: RNE ties
+    rows.append(row([ties] * nb))
+    rows.append(row([rng.normal(0, 1e-38, 128).astype(np.float32)] * nb))      # subnormal amax
+    rows.append(row([rng.normal(0, 1e37, 128).astype(np.float32)] * nb))       # huge values
+    rows.append(row([np.where(np.arange(128) == 5, 1e-30, 1e-41).astype(np.float32)] * nb))
+    mix = []
+    for b in range(nb):
+        v = rng.normal(0, 10.0 ** rng.integers(-20, 20), 128).astype(np.float32)
+        v[rng.integers(0, 128)] = 0.0
+        mix.append(v)
+    rows.append(row(mix))
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    # every bf16 bit pattern that is finite, in blocks with a common amax
+    pats = np.arange(65536, dtype=np.uint32)
+    fin = pats[((pats >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    allb = torch.from_numpy(fin.view(np.int16)).view(torch.bfloat16)
+    n = (allb.numel() // H) * H
+    x = torch.cat([x, allb[:n].view(-1, H)])
+    return x
+
+
+def test_dispatch_adversarial_blocks():
+    x = adversarial_rows()
+    T, H, k = x.shape[0], x.shape[1], 3
+    cfg = CONFIGS["v3"].scaled(T)
+    rng = np.random.default_rng(13)
+    slot = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    from combine_ep_route_02_b200 import ep_dispatch
+    rx = torch.empty((T * k, H), dtype=torch.uint8, device="cuda")
+    rs = torch.empty((T * k, H // 128), dtype=torch.float32, device="cuda")
+    ep_dispatch(x.cuda(), T, H, k, torch.from_numpy(slot).cuda(), True, rx, rs)
+    torch.cuda.synchronize()
+    ref_x, ref_s = oracle.dispatch(x, slot, True)
+    assert np.array_equal(rx.cpu().numpy(), ref_x)
+    assert np.array_equal(rs.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    assert cfg.T == T
+
+
+@pytest.mark.parametrize("num_sms", [1, 3, 37, 0])
+def test_dispatch_num_sms_and_invalid_slots(num_sms):
+    cfg = CONFIGS["ds16b"].scaled(517)
+    wl = Workload(cfg, seed=5)
+    idx, _, _ = oracle_route(cfg, wl)
+    lay = oracle_layout(cfg, wl, idx)
+    slot = lay["slot"].copy()
+    slot[3, 1] = -1                 # skipped
+    slot[10, 0] = cfg.T * cfg.topk  # out of range: skipped
+    path = make_path(cfg, wl, num_sms=num_sms)
+    path.recv_x.view(torch.uint8).fill_(0xAB)
+    path.recv_scale.fill_(-1.0)
+    path.slot.copy_(torch.from_numpy(slot))
+    path.dispatch(wl.x.cuda())
+    torch.cuda.synchronize()
+    rx, rs = oracle.dispatch(wl.x, slot, True)
+    got = path.recv_x.view(torch.uint8).cpu().numpy()
+    gs = path.recv_scale.cpu().numpy()
+    unwritten = np.setdiff1d(np.arange(cfg.T * cfg.topk), slot[slot >= 0][slot[slot >= 0] < cfg.T * cfg.topk])
+    written = np.setdiff1d(np.arange(cfg.T * cfg.topk), unwritten)
+    assert np.array_equal(got[written], rx[written])
+    assert np.array_equal(gs[written], rs[written])
+    assert (got[unwritten] == 0xAB).all() and (gs[unwritten] == -1.0).all()
+
+
+def test_dispatch_bf16_ragged():
+    cfg = CONFIGS["tiny"].scaled(333)
+    wl = Workload(cfg, seed=9)
+    idx, _, _ = oracle_route(cfg, wl)
+    lay = oracle_layout(cfg, wl, idx)
+    path = make_path(cfg, wl, num_sms=5)
+    path.slot.copy_(torch.from_numpy(lay["slot"]))
+    path.dispatch(wl.x.cuda())
+    torch.cuda.synchronize()
+    check_dispatch(cfg, wl.x, lay["slot"], path)
+
+
+# ---------------------------------------------------------------------------
+# combine
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ALL)
+def test_combine_full_size(name):
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    idx, w, _ = oracle_route(cfg, wl)
+    lay = oracle_layout(cfg, wl, idx)
+    y = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=1)
+    path = make_path(cfg, wl)
+    path.slot.copy_(torch.from_numpy(lay["slot"]))
+    path.topk_w.copy_(torch.from_numpy(w))
+    path.combine(y)
+    torch.cuda.synchronize()
+    ref = oracle.combine(y.cpu(), lay["slot"], w)
+    got = u16(path.out)
+    assert_combine_close(got, ref)
+    # same rounding sequence as the oracle: expected bit-identical
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("k", [1, 3, 8, 9, 17, 32])
+def test_combine_topk_and_invalid_slots(k):
+    rng = np.random.default_rng(20 + k)
+    T, H = 257, 520
+    y = device_normal_bf16(T * k, H, seed=k)
+    slot = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    slot[0, 0] = -1
+    slot[7, k - 1] = T * k
+    w = rng.uniform(-1, 2, (T, k)).astype(np.float32)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    from combine_ep_route_02_b200 import ep_combine
+    ep_combine(y, torch.from_numpy(slot).cuda(), torch.from_numpy(w).cuda(), T, H, k, out,
+               num_sms=7)
+    torch.cuda.synchronize()
+    ref = oracle.combine(y.cpu(), slot, w)
+    assert_combine_close(u16(out), ref)
+    assert np.array_equal(u16(out), ref)
+
+
+# ---------------------------------------------------------------------------
+# whole path
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["v3", "skew", "v3_decode"])
+def test_full_path(name):
+    """route -> layout -> dispatch -> combine in one stream, as the bench runs it"""
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    path = make_path(cfg, wl)
+    y = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=2)
+    path.step(wl.x.cuda(), wl.logits.cuda(), wl.bias.cuda(), y)
+    torch.cuda.synchronize()
+    idx, w, hard = oracle_route(cfg, wl)
+    assert hard.sum() == 0
+    assert np.array_equal(path.topk_idx.cpu().numpy(), idx)
+    assert np.array_equal(path.topk_w.cpu().numpy().view(np.uint32), w.view(np.uint32))
+    lay = oracle_layout(cfg, wl, idx)
+    got = gpu_layout_dict(path)
+    for n in LAYOUT_FIELDS:
+        assert np.array_equal(got[n].reshape(lay[n].shape), lay[n]), n
+    check_dispatch(cfg, wl.x, lay["slot"], path)
+    ref = oracle.combine(y.cpu(), lay["slot"], w)
+    assert_combine_close(u16(path.out), ref)
+
+
+def test_identity_expert_round_trip():
+    """dispatch -> dequantised identity experts -> combine recovers x"""
+    cfg = CONFIGS["ds16b"]
+    wl = Workload(cfg)
+    path = make_path(cfg, wl)
+    x = wl.x.cuda()
+    path.route(wl.logits.cuda(), wl.bias.cuda())
+    path.layout()
+    path.dispatch(x)
+    deq = path.recv_x.float() * path.recv_scale.repeat_interleave(128, dim=1)
+    path.combine(deq.to(torch.bfloat16))
+    torch.cuda.synchronize()
+    xf = x.double()
+    sc = xf.abs().view(cfg.T, -1, 128).amax(2).repeat_interleave(128, dim=1) / 448
+    bound = (2.0 ** -4 + 2.0 ** -7) * xf.abs() + 2.0 ** -9 * sc + 1e-30
+    assert ((path.out.double() - xf).abs() <= bound).all()
+
+
+def test_deterministic_across_runs_and_grids():
+    cfg = CONFIGS["skew"].scaled(3000)
+    wl = Workload(cfg, seed=4)
+    y = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=3)
+    outs = []
+    for num_sms in (0, 11):
+        path = make_path(cfg, wl, num_sms=num_sms)
+        path.step(wl.x.cuda(), wl.logits.cuda(), wl.bias.cuda(), y)
+        torch.cuda.synchronize()
+        outs.append([t.cpu().clone() for t in (path.topk_idx, path.slot, path.src,
+                                                path.recv_x.view(torch.uint8), path.recv_scale,
+                                                path.out)])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
