@@ -20,6 +20,7 @@ oracle on the host cores on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import os
 import statistics
@@ -72,12 +73,11 @@ class ClockSampler:
         try:
             import pynvml
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id \
-                if hasattr(torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
-            if bus:
-                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
-            else:
-                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            props = torch.cuda.get_device_properties(device_index)
+            # NVML wants the textual bus id; torch gives its three integers
+            bus = "%08X:%02X:%02X.0" % (int(props.pci_domain_id), int(props.pci_bus_id),
+                                        int(props.pci_device_id))
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
             self.nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
@@ -190,6 +190,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
+    faulthandler.enable()
     cfg = CONFIGS[args.config]
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
