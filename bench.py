@@ -262,6 +262,7 @@ def main():
     K = args.steps
     c0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
     c1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
+    l0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
     d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
     d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
     s0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -278,6 +279,7 @@ def main():
         s0[i].record(stream)
         if kev:
             path.route(lg, bias)
+            l0[i].record(stream)
             path.layout()
             d0[i].record(stream)
             path.dispatch(x)
@@ -316,7 +318,10 @@ def main():
                     if peak_kind == "measured" else "fallback 6650 GB/s",
                     "traffic": None}
         dc_ms = comb_ms + disp_ms
+        route_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(s0, l0))
+        layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(l0, d0))
         extra = {
+            "route_us": route_ms * 1e3, "layout_us": layout_ms * 1e3,
             "dispatch_us": disp_ms * 1e3, "combine_us": comb_ms * 1e3,
             "dispatch_gbs": disp_gbs, "combine_gbs": comb_gbs,
             "dispatch_combine_tokens_per_s": cfg.T * world / (dc_ms * 1e-3),
