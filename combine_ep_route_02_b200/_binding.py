@@ -26,7 +26,7 @@ EP_DEV_BAD_REPLICA = 2
 
 # every symbol declared in include/ep.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
-           "ep_combine", "ep_status_string")
+           "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc")
 
 
 class EpError(RuntimeError):
@@ -63,6 +63,9 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch.restype = I
         L.ep_combine.argtypes = [P, P, P, I, I, I, P, I, P]
         L.ep_combine.restype = I
+        L.ep_dispatch_layout_noalloc.argtypes = [P, I, I, I, I, I, P, P, I,
+                                                 P, P, P, P, P, P, P, P, P, P]
+        L.ep_dispatch_layout_noalloc.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -118,3 +121,14 @@ def ep_dispatch(x, T, H, k, slot, fp8, recv_x, recv_scale, num_sms=0, stream=Non
 def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, stream=None):
     _check("ep_combine", lib().ep_combine(_ptr(y), _ptr(slot), _ptr(topk_w), T, H, k,
                                           _ptr(out), num_sms, _stream(stream)))
+
+
+def ep_dispatch_layout_noalloc(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
+                               expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
+                               dev_status, stream=None):
+    """ep_dispatch_layout with the library's fixed device scratch instead of a
+    caller-provided workspace (for callers that cannot allocate device memory)."""
+    _check("ep_dispatch_layout_noalloc", lib().ep_dispatch_layout_noalloc(
+        _ptr(topk_idx), T, k, E, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
+        _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank), _ptr(rank_off), _ptr(tok_rank),
+        _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(dev_status), _stream(stream)))

@@ -184,6 +184,36 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *sl
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T,
                      int H, int k, void *out_bf16, int num_sms, ep_stream_t stream);
 
+/*
+ * Allocation-free variant of ep_dispatch_layout.  It has no counterpart in
+ * the pages; it exists for callers that cannot allocate device memory where
+ * they call the layout: code running inside another runtime's enqueue hook
+ * (an inference-engine plugin, a framework operator without access to its
+ * caching allocator), or a latency-bound decode step that cannot afford the
+ * device-wide synchronisation cudaMalloc may cause.
+ *
+ * Arguments and results are those of ep_dispatch_layout without
+ * `workspace`: the scratch lives in a fixed __device__ array of
+ * EP_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library keeps until the process exits.  Sizes whose
+ * ep_workspace_size(T, k, P, R) exceeds that limit return
+ * EP_ERR_UNSUPPORTED (with P = 256 and R = 8 that is about 250K tokens).
+ * The first call on each device looks up the array's device address (host
+ * code cannot use the array's name as a device pointer); make that first
+ * call before any stream capture.  The call allocates and frees nothing.
+ * All calls on a device share the one array and it keeps the last call's
+ * contents (the kernels need none of them cleared): calls whose work can
+ * overlap on the GPU (different streams, or several host threads) race on
+ * it and must be serialised by the caller.
+ */
+#define EP_NOALLOC_SCRATCH_BYTES (4u << 20)
+ep_status ep_dispatch_layout_noalloc(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                                     const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                                     int32_t *cnt_expert, int32_t *expert_off,
+                                     int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                                     uint8_t *in_rank, int32_t *slot, int32_t *src,
+                                     int32_t *dev_status, ep_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *ep_status_string(ep_status status);
 
