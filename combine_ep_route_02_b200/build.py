@@ -21,8 +21,8 @@ LIB = os.path.join(LIB_DIR, "libep_b200.so")
 HEADER = os.path.join(ROOT, "include", "ep.h")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
-              "--shared", "-Xptxas", "-warn-spills"]
+COMPILE_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
+                 "-Xptxas", "-warn-spills"]
 
 
 def nvcc() -> str:
@@ -43,16 +43,36 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+# Per-file compiler options (none needed at present).
+PER_FILE = {}
+
+BUILD_DIR = os.path.join(PKG, "_build")
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    tag = f"{os.getpid()}"
+    procs, objs = [], []
+    for src in sources():
+        name = os.path.basename(src)
+        obj = os.path.join(BUILD_DIR, name[:-3] + f".{tag}.o")
+        cmd = [nvcc(), *ARCH, *COMPILE_FLAGS, *PER_FILE.get(name, []), *extra,
+               "-c", src, "-o", obj]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((subprocess.Popen(cmd), cmd))
+        objs.append(obj)
+    failed = [cmd for p, cmd in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    tmp = LIB + f".tmp{tag}"
+    subprocess.check_call([nvcc(), *ARCH, "--shared", "-o", tmp, *objs])
+    for o in objs:
+        os.remove(o)
     os.replace(tmp, LIB)
     return LIB
 

@@ -25,11 +25,11 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ slot,
 {
     const int cpr = H >> 3;
     const long long total = (long long)T * cpr;
-    const long long stride = (long long)gridDim.x * COMBINE_THREADS;
-    for (long long g = (long long)blockIdx.x * COMBINE_THREADS + threadIdx.x; g < total;
-         g += stride) {
-        const int t = (int)(g / cpr);
-        const int c = (int)(g - (long long)t * cpr);
+    const long long g0 = (long long)blockIdx.x * COMBINE_THREADS + threadIdx.x;
+    if (g0 >= total) return;
+    ChunkWalk it(g0, (long long)gridDim.x * COMBINE_THREADS, cpr);
+    for (; it.t < T; it.next()) {
+        const int t = it.t, c = it.c;
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
@@ -45,6 +45,8 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ slot,
                 wj[u] = ok[u] ? __ldg(w + (size_t)t * k + j) : 0.0f;
                 v[u] = ok[u] ? ld_stream(y + (size_t)s * H + (size_t)c * 8) : make_uint4(0, 0, 0, 0);
             }
+            // fp32 accumulation in j order: acc = RN(acc + RN(w * y)); the
+            // _rn intrinsics are never fused into an FMA
 #pragma unroll
             for (int u = 0; u < COMBINE_BATCH; ++u) {
                 if (!ok[u]) continue;

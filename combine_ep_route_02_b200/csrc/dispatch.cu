@@ -20,12 +20,40 @@ namespace {
 
 constexpr int DISPATCH_THREADS = 256;
 
-EP_DEV uint32_t quant4(const float *v, float scale)
+// fp32(x / scale), rounded to nearest even, from the block's shared
+// reciprocal rcp = fp32(1 / scale): one product, then Markstein's correction
+// step (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): the residual
+// x - q0 * scale is exact in one FMA and q0 + residual * rcp rounds to the
+// correctly rounded quotient.  Used only for normal scales with a normal
+// reciprocal (see fast_div_ok); the exhaustive dispatch test checks every
+// bf16 (x, amax) pair against the oracle's IEEE division.
+EP_DEV float div_by_scale(float x, float scale, float rcp)
 {
-    // q = e4m3(fp32(x / scale)), IEEE division rounded to nearest even
-    const uint32_t a = pack_e4m3x2(__fdiv_rn(v[0], scale), __fdiv_rn(v[1], scale));
-    const uint32_t b = pack_e4m3x2(__fdiv_rn(v[2], scale), __fdiv_rn(v[3], scale));
-    return a | (b << 16);
+    const float q0 = __fmul_rn(x, rcp);
+    const float r = __fmaf_rn(-q0, scale, x);
+    // scale > 0, so the quotient carries the sign of x; the correction
+    // would turn x = -0 into +0 (r = +0, then +0 + -0 = +0)
+    return copysignf(__fmaf_rn(r, rcp, q0), x);
+}
+
+// The correction is exact while the residual cannot underflow: for a
+// quotient large enough to reach an e4m3 rounding point (>= 2^-11) the
+// residual is about 2^-23 |x| >= 2^-34 scale, a normal number once
+// scale >= 2^-90; smaller quotients encode to zero either way.  Tinier
+// scales (amax below about 3.6e-25) take the IEEE division.
+EP_DEV bool fast_div_ok(float scale)
+{
+    return scale >= 0x1p-90f && scale <= 0x1p125f;
+}
+
+EP_DEV uint32_t quant4(const float *v, float scale, float rcp, bool fast)
+{
+    // q = e4m3(fp32(x / scale))
+    float q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = fast ? div_by_scale(v[i], scale, rcp) : __fdiv_rn(v[i], scale);
+    return pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
 }
 
 __global__ void __launch_bounds__(DISPATCH_THREADS)
@@ -39,14 +67,14 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
     const long long stride = (long long)gridDim.x * DISPATCH_THREADS;
     // the loop bound is block-uniform so every lane reaches the shuffles;
     // total is a multiple of 8, so a lane octet is all active or all idle
-    for (long long base = (long long)blockIdx.x * DISPATCH_THREADS; base < total; base += stride) {
-        const long long g = base + threadIdx.x;
-        const bool active = g < total;
-        int t = 0, c = 0;
+    const long long g0 = (long long)blockIdx.x * DISPATCH_THREADS + threadIdx.x;
+    ChunkWalk it(g0, stride, cpr);
+    for (long long base = (long long)blockIdx.x * DISPATCH_THREADS; base < total;
+         base += stride, it.next()) {
+        const bool active = it.t < T;
+        const int t = it.t, c = it.c;
         uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
         if (active) {
-            t = (int)(g / cpr);
-            c = (int)(g - (long long)t * cpr);
             const uint16_t *p = x + (size_t)t * H + (size_t)c * 16;
             lo = ld_stream(p);
             hi = ld_stream(p + 8);
@@ -71,10 +99,12 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
 
         uint4 q = make_uint4(0, 0, 0, 0);  // amax == 0: scale 0, zero bytes
         if (amax != 0.0f) {
-            q.x = quant4(v + 0, scale);
-            q.y = quant4(v + 4, scale);
-            q.z = quant4(v + 8, scale);
-            q.w = quant4(v + 12, scale);
+            const bool fast = fast_div_ok(scale);
+            const float rcp = fast ? __frcp_rn(scale) : 0.0f;
+            q.x = quant4(v + 0, scale, rcp, fast);
+            q.y = quant4(v + 4, scale, rcp, fast);
+            q.z = quant4(v + 8, scale, rcp, fast);
+            q.w = quant4(v + 12, scale, rcp, fast);
         }
         if (active) {
             const int32_t *sl = slot + (size_t)t * k;
@@ -95,11 +125,11 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
 {
     const int cpr = H >> 3;  // 8-element (16-byte) chunks per row
     const long long total = (long long)T * cpr;
-    const long long stride = (long long)gridDim.x * DISPATCH_THREADS;
-    for (long long g = (long long)blockIdx.x * DISPATCH_THREADS + threadIdx.x; g < total;
-         g += stride) {
-        const int t = (int)(g / cpr);
-        const int c = (int)(g - (long long)t * cpr);
+    const long long g0 = (long long)blockIdx.x * DISPATCH_THREADS + threadIdx.x;
+    if (g0 >= total) return;
+    ChunkWalk it(g0, (long long)gridDim.x * DISPATCH_THREADS, cpr);
+    for (; it.t < T; it.next()) {
+        const int t = it.t, c = it.c;
         const uint4 v = ld_stream(x + (size_t)t * H + (size_t)c * 8);
         const int32_t *sl = slot + (size_t)t * k;
         for (int j = 0; j < k; ++j) {

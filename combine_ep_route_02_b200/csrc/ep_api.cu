@@ -122,7 +122,7 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *sl
     if (T < 0 || H < 1 || k < 1) return EP_ERR_INVALID;
     if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
-    if ((long long)T * k >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
     if (T > 0 && (!x_bf16 || !slot || !recv_x || (fp8 && !recv_scale))) return EP_ERR_INVALID;
     if (!aligned(x_bf16, 16) || !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(slot, 4))
         return EP_ERR_INVALID;
@@ -136,7 +136,7 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
 {
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
-    if ((long long)T * k >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
     if (T > 0 && (!y_bf16 || !slot || !topk_w || !out_bf16)) return EP_ERR_INVALID;
     if (!aligned(y_bf16, 16) || !aligned(out_bf16, 16) || !aligned(slot, 4) || !aligned(topk_w, 4))
         return EP_ERR_INVALID;

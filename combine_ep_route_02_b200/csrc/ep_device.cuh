@@ -56,6 +56,24 @@ EP_DEV uint32_t pack_e4m3x2(float lo, float hi)
     return r;
 }
 
+// Walks a flat chunk index g = t * cpr + c forward by a fixed stride without
+// dividing in the loop: one division when the walk starts.
+struct ChunkWalk {
+    int t, c, st, sc, cpr;
+    EP_DEV ChunkWalk(long long g0, long long stride, int cpr_)
+        : t((int)(g0 / cpr_)), c((int)(g0 % cpr_)), st((int)(stride / cpr_)),
+          sc((int)(stride % cpr_)), cpr(cpr_) {}
+    EP_DEV void next()
+    {
+        c += sc;
+        t += st;
+        if (c >= cpr) {
+            c -= cpr;
+            ++t;
+        }
+    }
+};
+
 // (value desc, index asc) total order used by every selection.
 EP_DEV bool beats(float va, int ia, float vb, int ib)
 {

@@ -2,9 +2,18 @@
 //
 // DeepSeek group-limited routing (DeepSeek Open Infra day-4 summary, EPLB
 // section) with plain top-k as its one-group special case (Perplexity blog,
-// section "MoE Router").  Lane l holds experts [l*EPL, (l+1)*EPL); the group
-// scores, the group choice and each of the k expert choices are warp-shuffle
-// reductions, so no sort and no shared memory is needed.
+// section "MoE Router").  Lane l holds experts [l*EPL, (l+1)*EPL).
+//
+// Every arg-max (groups, then each of the k experts) is two warp reductions
+// on integers: redux.sync max over an order-preserving 32-bit image of the
+// fp32 key, then redux.sync min over the indices of the lanes holding that
+// maximum, which is exactly the (key desc, index asc) order.  Keys are never
+// -0.0 or NaN here (s >= 0, and s + b rounds an exact zero to +0), so the
+// integer order equals the fp32 order.
+//
+// When a group is a power-of-two number of whole lanes (E/G a multiple of
+// EPL), each lane sits in one group and the group top-2 is a butterfly over
+// that group's lanes only; otherwise a general loop over groups is used.
 #include <math.h>
 
 #include "ep_device.cuh"
@@ -13,6 +22,24 @@
 namespace ep {
 
 namespace {
+
+// fp32 -> uint32 with the same order (for finite, non-NaN values; -0 and +0
+// map to different images, which never matters for the keys used here).
+EP_DEV uint32_t ordered(float f)
+{
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+constexpr uint32_t NONE = 0u;  // below the image of every float, -inf included
+
+// winner of (key desc, index asc) over the warp; every lane gets it
+EP_DEV int warp_pick(uint32_t key, int idx)
+{
+    const uint32_t kmax = __reduce_max_sync(FULL_MASK, key);
+    const uint32_t cand = (key == kmax) ? (uint32_t)idx : 0xffffffffu;
+    return (int)__reduce_min_sync(FULL_MASK, cand);
+}
 
 template <int EPL>
 __global__ void __launch_bounds__(256)
@@ -24,10 +51,21 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
     const int warps = gridDim.x * (blockDim.x >> 5);
     const int e0 = lane * EPL;
     const int gs = E / G;
+    // each lane lies inside one group when gs is a multiple of EPL; the
+    // butterfly below also needs the group's lane count to be a power of two
+    const int lpg = gs / EPL;
+    const bool aligned = (gs % EPL) == 0 && (lpg & (lpg - 1)) == 0;
+    const int lanes_per_group = aligned ? lpg : 0;
+    const int my_group = (e0 < E) ? e0 / gs : -1;        // valid when aligned
 
     float b[EPL];
+    int gid[EPL];  // token-invariant group of each held expert (-1: none)
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) b[i] = (bias != nullptr && e0 + i < E) ? bias[e0 + i] : 0.0f;
+    for (int i = 0; i < EPL; ++i) {
+        const bool v = e0 + i < E;
+        b[i] = (bias != nullptr && v) ? bias[e0 + i] : 0.0f;
+        gid[i] = v ? (e0 + i) / gs : -1;
+    }
 
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
         const float *row = logits + (size_t)t * E;
@@ -50,31 +88,61 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
         }
 
         // s = fp32(1 / (1 + exp(-x))) evaluated in fp64; key = fp32(s + b)
-        float s[EPL], key[EPL];
-        unsigned excluded = 0;  // bit i: expert e0+i is not eligible
+        float s[EPL];
+        uint32_t key[EPL];
+        uint32_t live = 0;  // bit i: expert e0+i exists and is still eligible
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             if (e0 + i < E) {
                 s[i] = __double2float_rn(1.0 / (1.0 + exp(-(double)x[i])));
-                key[i] = __fadd_rn(s[i], b[i]);
+                key[i] = ordered(__fadd_rn(__fadd_rn(s[i], b[i]), 0.0f));
+                live |= 1u << i;
             } else {
                 s[i] = 0.0f;
-                key[i] = -INFINITY;
-                excluded |= 1u << i;
+                key[i] = NONE;
             }
         }
 
         if (G > 1) {
-            // group score = fp32 sum of the two largest keys in the group;
-            // lane g keeps the score of group g
-            float my_score = -INFINITY;
-            for (int g = 0; g < G; ++g) {
+            // group score = fp32 sum of the two largest keys in the group
+            uint32_t chosen = 0;
+            if (aligned) {
                 float a1 = -INFINITY, a2 = -INFINITY;
 #pragma unroll
                 for (int i = 0; i < EPL; ++i) {
-                    const int e = e0 + i;
-                    if (e < E && e / gs == g) {
-                        const float v = key[i];
+                    if (!((live >> i) & 1u)) continue;
+                    const float v = __fadd_rn(s[i], b[i]);
+                    if (v > a1) {
+                        a2 = a1;
+                        a1 = v;
+                    } else if (v > a2) {
+                        a2 = v;
+                    }
+                }
+                // butterfly over the lanes of this group (they are contiguous
+                // and start at a multiple of lanes_per_group)
+                for (int off = 1; off < lanes_per_group; off <<= 1) {
+                    const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                    const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                    const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                    a1 = fmaxf(a1, o1);
+                    a2 = n2;
+                }
+                const uint32_t my_score =
+                    (my_group >= 0) ? ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f)) : NONE;
+                for (int r = 0; r < Kg; ++r) {
+                    const bool cand = my_group >= 0 && !((chosen >> my_group) & 1u);
+                    const int g = warp_pick(cand ? my_score : NONE, cand ? my_group : 0x7fffffff);
+                    chosen |= 1u << g;
+                }
+            } else {
+                uint32_t my_score = NONE;  // lane g keeps the score of group g
+                for (int g = 0; g < G; ++g) {
+                    float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) {
+                        if (gid[i] != g) continue;
+                        const float v = __fadd_rn(s[i], b[i]);
                         if (v > a1) {
                             a2 = a1;
                             a1 = v;
@@ -82,60 +150,59 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
                             a2 = v;
                         }
                     }
-                }
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
-                    const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
-                    const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
-                    a1 = fmaxf(a1, o1);
-                    a2 = n2;
+                    for (int off = 16; off > 0; off >>= 1) {
+                        const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                        const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                        const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                        a1 = fmaxf(a1, o1);
+                        a2 = n2;
+                    }
+                    if (lane == g) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
                 }
-                if (lane == g) my_score = __fadd_rn(a1, a2);
-            }
-            // keep the Kg best groups, ties to the lower group id
-            unsigned chosen = 0;
-            for (int r = 0; r < Kg; ++r) {
-                const bool cand = lane < G && !((chosen >> lane) & 1u);
-                float v = cand ? my_score : -INFINITY;
-                int id = cand ? lane : 0x7fffffff;
-                warp_argmax(v, id);
-                chosen |= 1u << id;
+                for (int r = 0; r < Kg; ++r) {
+                    const bool cand = lane < G && !((chosen >> lane) & 1u);
+                    const int g = warp_pick(cand ? my_score : NONE, cand ? lane : 0x7fffffff);
+                    chosen |= 1u << g;
+                }
             }
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = e0 + i;
-                if (e < E && !((chosen >> (e / gs)) & 1u)) excluded |= 1u << i;
-            }
+            for (int i = 0; i < EPL; ++i)
+                if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) live &= ~(1u << i);
         }
 
-        // k rounds of (key desc, index asc) arg-max over eligible experts
-        unsigned taken = excluded;
+        // lane-local best (lowest index among equal keys: strict >)
+        uint32_t best_k = NONE;
+        int best_i = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (((live >> i) & 1u) && (best_i == 0x7fffffff || key[i] > best_k)) {
+                best_k = key[i];
+                best_i = e0 + i;
+            }
+
         int sel_idx = 0;
         float sel_s = 0.0f;
         for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (!((taken >> i) & 1u) && beats(key[i], e0 + i, bv, bi)) {
-                    bv = key[i];
-                    bi = e0 + i;
-                }
-            warp_argmax(bv, bi);
-            const int owner = bi / EPL;  // k <= eligible count: bi is a real expert
+            const int e = warp_pick(best_i == 0x7fffffff ? NONE : best_k, best_i);
+            const int owner = e / EPL;  // k <= eligible experts, so e is real
             float sv = 0.0f;
             if (lane == owner) {
+                live &= ~(1u << (e - e0));
+                best_k = NONE;
+                best_i = 0x7fffffff;
 #pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (e0 + i == bi) {
-                        sv = s[i];
-                        taken |= 1u << i;
+                for (int i = 0; i < EPL; ++i) {
+                    if (e0 + i == e) sv = s[i];
+                    if (((live >> i) & 1u) && (best_i == 0x7fffffff || key[i] > best_k)) {
+                        best_k = key[i];
+                        best_i = e0 + i;
                     }
+                }
             }
             sv = __shfl_sync(FULL_MASK, sv, owner);
             if (lane == r) {
-                sel_idx = bi;
+                sel_idx = e;
                 sel_s = sv;
             }
         }
