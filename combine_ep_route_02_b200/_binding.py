@@ -23,6 +23,7 @@ EP_ERR_CUDA = 3
 EP_ERR_DEVICE = 4
 EP_DEV_BAD_EXPERT = 1
 EP_DEV_BAD_REPLICA = 2
+EP_DEV_TIMEOUT = 4
 
 # every symbol declared in include/ep.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
@@ -59,9 +60,9 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_layout.argtypes = [P, I, I, I, I, I, P, P, I,
                                          P, P, P, P, P, P, P, P, P, P, P]
         L.ep_dispatch_layout.restype = I
-        L.ep_dispatch.argtypes = [P, I, I, I, P, I, P, P, I, P]
+        L.ep_dispatch.argtypes = [P, I, I, I, P, I, P, P, I, P, P]
         L.ep_dispatch.restype = I
-        L.ep_combine.argtypes = [P, P, P, I, I, I, P, I, P]
+        L.ep_combine.argtypes = [P, P, P, I, I, I, P, I, P, P]
         L.ep_combine.restype = I
         L.ep_dispatch_layout_noalloc.argtypes = [P, I, I, I, I, I, P, P, I,
                                                  P, P, P, P, P, P, P, P, P, P]
@@ -112,15 +113,17 @@ def ep_dispatch_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_exp
         _stream(stream)))
 
 
-def ep_dispatch(x, T, H, k, slot, fp8, recv_x, recv_scale, num_sms=0, stream=None):
+def ep_dispatch(x, T, H, k, slot, fp8, recv_x, recv_scale, num_sms=0, dev_status=None,
+                stream=None):
     _check("ep_dispatch", lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot), int(bool(fp8)),
                                             _ptr(recv_x), _ptr(recv_scale), num_sms,
-                                            _stream(stream)))
+                                            _ptr(dev_status), _stream(stream)))
 
 
-def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, stream=None):
+def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, dev_status=None, stream=None):
     _check("ep_combine", lib().ep_combine(_ptr(y), _ptr(slot), _ptr(topk_w), T, H, k,
-                                          _ptr(out), num_sms, _stream(stream)))
+                                          _ptr(out), num_sms, _ptr(dev_status),
+                                          _stream(stream)))
 
 
 def ep_dispatch_layout_noalloc(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,

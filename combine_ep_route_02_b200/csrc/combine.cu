@@ -23,6 +23,8 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ slot,
                const float *__restrict__ w, int T, int H, int k, int n_rows,
                uint16_t *__restrict__ out)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int cpr = H >> 3;
     const long long total = (long long)T * cpr;
     const long long g0 = (long long)blockIdx.x * COMBINE_THREADS + threadIdx.x;
@@ -82,10 +84,9 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s)
     const long long chunks = (long long)a.T * (a.H / 8);
     long long blocks = (chunks + COMBINE_THREADS - 1) / COMBINE_THREADS;
     if (blocks > a.grid) blocks = a.grid;
-    combine_kernel<<<(int)blocks, COMBINE_THREADS, 0, s>>>(
-        static_cast<const uint16_t *>(a.y), a.slot, a.w, a.T, a.H, a.k, a.T * a.k,
-        static_cast<uint16_t *>(a.out));
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3((int)blocks), dim3(COMBINE_THREADS), 0, s,
+                      static_cast<const uint16_t *>(a.y), a.slot, a.w, a.T, a.H, a.k, a.T * a.k,
+                      static_cast<uint16_t *>(a.out));
 }
 
 }  // namespace ep

@@ -56,11 +56,49 @@ EP_DEV uint32_t quant4(const float *v, float scale, float rcp, bool fast)
     return pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
 }
 
+// Quantise one 16-element chunk (two 16-byte bf16 vectors).  The 8 lanes
+// whose chunks form one 128-element block must call this together (xor
+// shuffles over lane offsets 1, 2, 4); every lane of the warp must call it.
+EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
+{
+    float v[16];
+    v[0] = bf16_lo(lo.x);  v[1] = bf16_hi(lo.x);
+    v[2] = bf16_lo(lo.y);  v[3] = bf16_hi(lo.y);
+    v[4] = bf16_lo(lo.z);  v[5] = bf16_hi(lo.z);
+    v[6] = bf16_lo(lo.w);  v[7] = bf16_hi(lo.w);
+    v[8] = bf16_lo(hi.x);  v[9] = bf16_hi(hi.x);
+    v[10] = bf16_lo(hi.y); v[11] = bf16_hi(hi.y);
+    v[12] = bf16_lo(hi.z); v[13] = bf16_hi(hi.z);
+    v[14] = bf16_lo(hi.w); v[15] = bf16_hi(hi.w);
+
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 4));
+    const float scale = __fdiv_rn(amax, 448.0f);
+    scale_out = scale;
+
+    uint4 q = make_uint4(0, 0, 0, 0);  // amax == 0: scale 0, zero bytes
+    if (amax != 0.0f) {
+        const bool fast = fast_div_ok(scale);
+        const float rcp = fast ? __frcp_rn(scale) : 0.0f;
+        q.x = quant4(v + 0, scale, rcp, fast);
+        q.y = quant4(v + 4, scale, rcp, fast);
+        q.z = quant4(v + 8, scale, rcp, fast);
+        q.w = quant4(v + 12, scale, rcp, fast);
+    }
+    return q;
+}
+
 __global__ void __launch_bounds__(DISPATCH_THREADS)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                     const int32_t *__restrict__ slot, uint8_t *__restrict__ recv_x,
                     float *__restrict__ recv_scale, int n_rows)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int cpr = H >> 4;  // 16-element chunks per row (a multiple of 8)
     const int S = H >> 7;
     const long long total = (long long)T * cpr;
@@ -79,33 +117,8 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
             lo = ld_stream(p);
             hi = ld_stream(p + 8);
         }
-        float v[16];
-        v[0] = bf16_lo(lo.x);  v[1] = bf16_hi(lo.x);
-        v[2] = bf16_lo(lo.y);  v[3] = bf16_hi(lo.y);
-        v[4] = bf16_lo(lo.z);  v[5] = bf16_hi(lo.z);
-        v[6] = bf16_lo(lo.w);  v[7] = bf16_hi(lo.w);
-        v[8] = bf16_lo(hi.x);  v[9] = bf16_hi(hi.x);
-        v[10] = bf16_lo(hi.y); v[11] = bf16_hi(hi.y);
-        v[12] = bf16_lo(hi.z); v[13] = bf16_hi(hi.z);
-        v[14] = bf16_lo(hi.w); v[15] = bf16_hi(hi.w);
-
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 4));
-        const float scale = __fdiv_rn(amax, 448.0f);
-
-        uint4 q = make_uint4(0, 0, 0, 0);  // amax == 0: scale 0, zero bytes
-        if (amax != 0.0f) {
-            const bool fast = fast_div_ok(scale);
-            const float rcp = fast ? __frcp_rn(scale) : 0.0f;
-            q.x = quant4(v + 0, scale, rcp, fast);
-            q.y = quant4(v + 4, scale, rcp, fast);
-            q.z = quant4(v + 8, scale, rcp, fast);
-            q.w = quant4(v + 12, scale, rcp, fast);
-        }
+        float scale;
+        const uint4 q = quant_chunk(lo, hi, scale);
         if (active) {
             const int32_t *sl = slot + (size_t)t * k;
             for (int j = 0; j < k; ++j) {
@@ -123,6 +136,8 @@ __global__ void __launch_bounds__(DISPATCH_THREADS)
 dispatch_bf16_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                      const int32_t *__restrict__ slot, uint16_t *__restrict__ recv_x, int n_rows)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int cpr = H >> 3;  // 8-element (16-byte) chunks per row
     const long long total = (long long)T * cpr;
     const long long g0 = (long long)blockIdx.x * DISPATCH_THREADS + threadIdx.x;
@@ -139,7 +154,153 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
     }
 }
 
+// ---------------------------------------------------------------------------
+// FP8 dispatch with TMA bulk copies (rows whose scale row is a whole number of
+// 16-byte units, H % 512 == 0).  A persistent CTA walks tokens
+// t = blockIdx.x, blockIdx.x + gridDim.x, ...:
+//   - thread 0 keeps TMA_IN_STAGES row loads (2H bytes each) in flight into
+//     shared memory, each completing on its own mbarrier;
+//   - all threads quantise the row from shared memory into an output stage
+//     (H code bytes + H/128 fp32 scales);
+//   - lanes j < k of warp 0 each send the stage to receive row slot[t, j]
+//     with two bulk stores and track them in their own bulk groups, so an
+//     output stage is reused only after its previous stores have read it.
+// Memory traffic is issued by the TMA engine, so the threads' own loads and
+// stores no longer bound the number of bytes in flight.
+// ---------------------------------------------------------------------------
+constexpr int TMA_IN_STAGES = 4;
+constexpr int TMA_OUT_STAGES = 4;
+constexpr uint32_t TMA_WAIT_LIMIT = 1u << 22;  // polls before reporting a timeout
+constexpr int DEV_TIMEOUT = 4;                 // EP_DEV_TIMEOUT
+
+__host__ __device__ inline size_t tma_smem_bytes(int H)
+{
+    return (size_t)TMA_IN_STAGES * 2 * H + (size_t)TMA_OUT_STAGES * (H + H / 32) +
+           TMA_IN_STAGES * sizeof(uint64_t);
+}
+
+__global__ void __launch_bounds__(512)
+dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
+                        const int32_t *__restrict__ slot, uint8_t *__restrict__ recv_x,
+                        float *__restrict__ recv_scale, int n_rows, int32_t *dev_status)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int S = H >> 7;
+    const uint32_t in_bytes = 2u * (uint32_t)H;
+    const uint32_t in_base = smem_u32(smem);
+    const uint32_t q_base = in_base + TMA_IN_STAGES * in_bytes;
+    const uint32_t sc_base = q_base + TMA_OUT_STAGES * (uint32_t)H;
+    const uint32_t bar_base = sc_base + TMA_OUT_STAGES * (uint32_t)S * 4u;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int first = blockIdx.x, step = gridDim.x;
+    const int n_my = (first < T) ? (T - first + step - 1) / step : 0;
+
+    pdl_launch_dependents();
+    if (tid == 0) {
+        for (int st = 0; st < TMA_IN_STAGES; ++st) mbar_init(bar_base + 8 * st, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();
+
+    if (tid == 0)
+        for (int st = 0; st < TMA_IN_STAGES && st < n_my; ++st) {
+            const int t = first + st * step;
+            mbar_arrive_expect_tx(bar_base + 8 * st, in_bytes);
+            bulk_load(in_base + st * in_bytes, x + (size_t)t * H, in_bytes, bar_base + 8 * st);
+        }
+
+    const int cpr = H >> 4;
+    int failed_at = -1;
+    for (int it = 0; it < n_my; ++it) {
+        const int t = first + it * step;
+        const int st = it % TMA_IN_STAGES;
+        const int o = it % TMA_OUT_STAGES;
+        int my_slot = -1;
+        if (warp == 0 && lane < k) my_slot = __ldg(slot + (size_t)t * k + lane);
+        const bool ok = mbar_wait(bar_base + 8 * st, (it / TMA_IN_STAGES) & 1, TMA_WAIT_LIMIT);
+        if (!__syncthreads_and(ok)) {
+            failed_at = it;
+            break;
+        }
+        const uint32_t in = in_base + st * in_bytes;
+        const uint32_t qo = q_base + o * (uint32_t)H;
+        const uint32_t so = sc_base + o * (uint32_t)S * 4u;
+        // cpr is a multiple of 8 and the bound is block-uniform, so every lane
+        // reaches the shuffles and lane octets are all active or all idle
+        for (int c0 = 0; c0 < cpr; c0 += blockDim.x) {
+            const int c = c0 + tid;
+            const bool act = c < cpr;
+            uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+            if (act) {
+                lo = lds128(in + 32u * c);
+                hi = lds128(in + 32u * c + 16u);
+            }
+            float scale;
+            const uint4 q = quant_chunk(lo, hi, scale);
+            if (act) {
+                sts128(qo + 16u * c, q);
+                if ((c & 7) == 0)
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(so + 4u * (c >> 3)), "f"(scale)
+                                 : "memory");
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();  // the input stage is consumed, the output stage written
+        if (warp == 0) {
+            if (lane == 0 && it + TMA_IN_STAGES < n_my) {
+                const int t2 = first + (it + TMA_IN_STAGES) * step;
+                mbar_arrive_expect_tx(bar_base + 8 * st, in_bytes);
+                bulk_load(in, x + (size_t)t2 * H, in_bytes, bar_base + 8 * st);
+            }
+            if (lane < k) {
+                if ((unsigned)my_slot < (unsigned)n_rows) {
+                    bulk_store(recv_x + (size_t)my_slot * H, qo, (uint32_t)H);
+                    bulk_store(recv_scale + (size_t)my_slot * S, so, (uint32_t)S * 4u);
+                }
+                bulk_commit();
+                // the stage written next iteration was sent TMA_OUT_STAGES-1
+                // groups ago: wait until those stores have read it
+                bulk_wait_read<TMA_OUT_STAGES - 1>();
+            }
+        }
+        __syncthreads();
+    }
+    if (warp == 0 && lane < k) bulk_wait_all();
+    if (failed_at >= 0 && tid == 0) {
+        // let the loads still in flight land before the CTA's shared memory
+        // goes away, then report
+        for (int it = failed_at; it < n_my && it < failed_at + TMA_IN_STAGES; ++it)
+            mbar_wait(bar_base + 8 * (it % TMA_IN_STAGES), (it / TMA_IN_STAGES) & 1, TMA_WAIT_LIMIT);
+        if (dev_status != nullptr) atomicOr(dev_status, DEV_TIMEOUT);
+    }
+}
+
+int tma_threads(int H)
+{
+    int t = ((H / 16 + 31) / 32) * 32;
+    if (t < 64) t = 64;
+    if (t > 512) t = 512;
+    return t;
+}
+
 }  // namespace
+
+bool dispatch_tma_ok(const DispatchArgs &a)
+{
+    return a.fp8 && a.H % 512 == 0 && tma_smem_bytes(a.H) <= 200 * 1024 &&
+           (reinterpret_cast<uintptr_t>(a.recv_scale) & 15) == 0 && a.k <= 32;
+}
+
+int dispatch_tma_blocks_per_sm(int H)
+{
+    const size_t smem = tma_smem_bytes(H);
+    cudaFuncSetAttribute(dispatch_fp8_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_fp8_tma_kernel, tma_threads(H), smem);
+    return n > 0 ? n : 1;
+}
 
 int dispatch_blocks_per_sm(int fp8)
 {
@@ -154,19 +315,24 @@ int dispatch_blocks_per_sm(int fp8)
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s)
 {
     if (a.T == 0) return cudaSuccess;
+    if (a.tma_grid > 0) {
+        const int blocks = a.T < a.tma_grid ? a.T : a.tma_grid;
+        return launch_pdl(dispatch_fp8_tma_kernel, dim3(blocks), dim3(tma_threads(a.H)),
+                          tma_smem_bytes(a.H), s, static_cast<const uint16_t *>(a.x), a.T, a.H,
+                          a.k, a.slot, static_cast<uint8_t *>(a.recv_x), a.recv_scale,
+                          a.T * a.k, a.dev_status);
+    }
     const long long chunks = (long long)a.T * (a.fp8 ? a.H / 16 : a.H / 8);
     long long blocks = (chunks + DISPATCH_THREADS - 1) / DISPATCH_THREADS;
     if (blocks > a.grid) blocks = a.grid;
     const int n_rows = a.T * a.k;
     if (a.fp8)
-        dispatch_fp8_kernel<<<(int)blocks, DISPATCH_THREADS, 0, s>>>(
-            static_cast<const uint16_t *>(a.x), a.T, a.H, a.k, a.slot,
-            static_cast<uint8_t *>(a.recv_x), a.recv_scale, n_rows);
-    else
-        dispatch_bf16_kernel<<<(int)blocks, DISPATCH_THREADS, 0, s>>>(
-            static_cast<const uint16_t *>(a.x), a.T, a.H, a.k, a.slot,
-            static_cast<uint16_t *>(a.recv_x), n_rows);
-    return cudaGetLastError();
+        return launch_pdl(dispatch_fp8_kernel, dim3((int)blocks), dim3(DISPATCH_THREADS), 0, s,
+                          static_cast<const uint16_t *>(a.x), a.T, a.H, a.k, a.slot,
+                          static_cast<uint8_t *>(a.recv_x), a.recv_scale, n_rows);
+    return launch_pdl(dispatch_bf16_kernel, dim3((int)blocks), dim3(DISPATCH_THREADS), 0, s,
+                      static_cast<const uint16_t *>(a.x), a.T, a.H, a.k, a.slot,
+                      static_cast<uint16_t *>(a.recv_x), n_rows);
 }
 
 }  // namespace ep

@@ -22,8 +22,6 @@ namespace {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
-
 ep_status from_cuda(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
 
 // grid of a streaming kernel: num_sms SMs (0 = all) x resident blocks per SM
@@ -43,6 +41,22 @@ int cached_blocks_per_sm(int which)
     if (dev < 64 && cache[dev][which] > 0) return cache[dev][which];
     const int n = which == 2 ? combine_blocks_per_sm() : dispatch_blocks_per_sm(which);
     if (dev < 64) cache[dev][which] = n;
+    return n;
+}
+
+// TMA dispatch CTAs per SM for row length H (depends on shared memory)
+int tma_blocks_per_sm(int H)
+{
+    static volatile int cache_h[64] = {0};
+    static volatile int cache_n[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && cache_h[dev] == H && cache_n[dev] > 0) return cache_n[dev];
+    const int n = dispatch_tma_blocks_per_sm(H);
+    if (dev < 64) {
+        cache_n[dev] = n;
+        cache_h[dev] = H;
+    }
     return n;
 }
 
@@ -68,8 +82,7 @@ const char *ep_status_string(ep_status s)
 size_t ep_workspace_size(int T, int k, int P, int R)
 {
     if (T < 0 || k < 1 || P < 1 || R < 1) return 0;
-    const size_t NT = (size_t)layout_tiles(T > 0 ? T : 1);
-    return align256(NT * (size_t)P * sizeof(int32_t)) + align256(NT * (size_t)R * sizeof(int32_t));
+    return layout_workspace_bytes(T, k, P, R);
 }
 
 ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
@@ -107,38 +120,44 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
     if (!aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(slot, 4) || !aligned(src, 4) ||
         !aligned(dev_status, 4))
         return EP_ERR_INVALID;
-    const int NT = layout_tiles(T);
-    int32_t *ws = static_cast<int32_t *>(workspace);
+    const int NT = layout_tiles(T, k, P);
+    char *ws = static_cast<char *>(workspace);
+    const size_t o1 = align256((size_t)NT * P * sizeof(int32_t));
+    const size_t o2 = o1 + align256((size_t)NT * R * sizeof(int32_t));
     LayoutArgs a{topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
                  cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
-                 ws, ws + align256((size_t)NT * P * sizeof(int32_t)) / sizeof(int32_t),
-                 dev_status};
+                 reinterpret_cast<int32_t *>(ws), reinterpret_cast<int32_t *>(ws + o1),
+                 reinterpret_cast<int32_t *>(ws + o2), dev_status, layout_tile_tokens(T, k, P), NT};
     return from_cuda(launch_layout(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
-                      void *recv_x, float *recv_scale, int num_sms, ep_stream_t stream)
+                      void *recv_x, float *recv_scale, int num_sms, int32_t *dev_status,
+                      ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1) return EP_ERR_INVALID;
     if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
     if (T > 0 && (!x_bf16 || !slot || !recv_x || (fp8 && !recv_scale))) return EP_ERR_INVALID;
-    if (!aligned(x_bf16, 16) || !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(slot, 4))
+    if (!aligned(x_bf16, 16) || !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(slot, 4) ||
+        !aligned(dev_status, 4))
         return EP_ERR_INVALID;
     DispatchArgs a{x_bf16, T, H, k, slot, fp8 != 0, recv_x, recv_scale,
-                   streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0))};
+                   streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0)), 0, dev_status};
+    if (T > 0 && dispatch_tma_ok(a)) a.tma_grid = streaming_grid(num_sms, tma_blocks_per_sm(H));
     return from_cuda(launch_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T, int H,
-                     int k, void *out_bf16, int num_sms, ep_stream_t stream)
+                     int k, void *out_bf16, int num_sms, int32_t *dev_status, ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
     if (T > 0 && (!y_bf16 || !slot || !topk_w || !out_bf16)) return EP_ERR_INVALID;
-    if (!aligned(y_bf16, 16) || !aligned(out_bf16, 16) || !aligned(slot, 4) || !aligned(topk_w, 4))
+    if (!aligned(y_bf16, 16) || !aligned(out_bf16, 16) || !aligned(slot, 4) || !aligned(topk_w, 4) ||
+        !aligned(dev_status, 4))
         return EP_ERR_INVALID;
     CombineArgs a{y_bf16, slot, topk_w, T, H, k, out_bf16,
                   streaming_grid(num_sms, cached_blocks_per_sm(2))};

@@ -7,8 +7,13 @@
 
 namespace ep {
 
-// Tokens per tile of the layout kernels.  The workspace size depends on it.
-constexpr int LAYOUT_TILE = 64;
+// Layout tiling.  A tile of tokens is one block of the count and slot
+// kernels.  Up to LAYOUT_FUSED_MAX_TILES tiles, the slot kernel sums the tile
+// histograms of its expert columns itself; above that a column-scan kernel
+// runs in between.  The workspace size depends on this tiling.
+constexpr int LAYOUT_MIN_TILE = 64;
+constexpr int LAYOUT_MAX_TILE = 512;
+constexpr int LAYOUT_FUSED_MAX_TILES = 64;
 constexpr int LAYOUT_THREADS = 256;
 constexpr int LAYOUT_WARPS = LAYOUT_THREADS / 32;
 constexpr int MAX_EXPERTS = 1024;   // logical experts (routing)
@@ -37,7 +42,10 @@ struct LayoutArgs {
     int32_t *slot, *src;
     int32_t *tile_cnt;  // workspace [NT][P]
     int32_t *tile_tok;  // workspace [NT][R]
+    int32_t *tile_bad;  // workspace [NT]: status bits found by each count block
     int32_t *dev_status;
+    int tile_tokens;    // TT
+    int n_tiles;        // NT
 };
 
 struct DispatchArgs {
@@ -47,7 +55,9 @@ struct DispatchArgs {
     int fp8;
     void *recv_x;
     float *recv_scale;
-    int grid;
+    int grid;          // register-path grid
+    int tma_grid;      // > 0: use the TMA pipeline with this many CTAs
+    int32_t *dev_status;
 };
 
 struct CombineArgs {
@@ -59,7 +69,55 @@ struct CombineArgs {
     int grid;
 };
 
-inline int layout_tiles(int T) { return (T + LAYOUT_TILE - 1) / LAYOUT_TILE; }
+// Tokens per tile: enough for at most LAYOUT_FUSED_MAX_TILES tiles, within
+// [LAYOUT_MIN_TILE, LAYOUT_MAX_TILE], and small enough that the slot kernel's
+// shared memory ((10 P + 1) ints of tables + tile_tokens * k ints of pair
+// ids) stays under 200 KB.
+inline int layout_tile_tokens(int T, int k, int P)
+{
+    int tt = (T + LAYOUT_FUSED_MAX_TILES - 1) / LAYOUT_FUSED_MAX_TILES;
+    if (tt < LAYOUT_MIN_TILE) tt = LAYOUT_MIN_TILE;
+    if (tt > LAYOUT_MAX_TILE) tt = LAYOUT_MAX_TILE;
+    int cap = (51200 - 10 * P - 1) / (k > 0 ? k : 1);
+    cap = (cap / 32) * 32;
+    if (cap < 32) cap = 32;
+    return tt < cap ? tt : cap;
+}
+inline int layout_tiles(int T, int k, int P)
+{
+    const int tt = layout_tile_tokens(T, k, P);
+    return (T + tt - 1) / tt;
+}
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+// workspace bytes: tile_cnt, tile_tok, tile_bad, each 256-byte aligned
+inline size_t layout_workspace_bytes(int T, int k, int P, int R)
+{
+    const size_t NT = (size_t)layout_tiles(T > 0 ? T : 1, k, P);
+    return align256(NT * P * sizeof(int32_t)) + align256(NT * R * sizeof(int32_t)) +
+           align256(NT * sizeof(int32_t));
+}
+
+// Programmatic dependent launch: every kernel of the path is launched with
+// programmatic stream serialisation, calls pdl_launch_dependents() so the
+// next kernel's launch can begin, and pdl_wait() before it touches global
+// memory, which returns once the previous kernel in the stream has finished
+// and its writes are visible.  Without the launch attribute both are no-ops.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
@@ -68,6 +126,8 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 
 // resident blocks per SM for each streaming kernel at its block size
 int dispatch_blocks_per_sm(int fp8);
+bool dispatch_tma_ok(const DispatchArgs &a);
+int dispatch_tma_blocks_per_sm(int H);
 int combine_blocks_per_sm();
 int device_sm_count();
 

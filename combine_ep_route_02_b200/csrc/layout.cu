@@ -8,16 +8,18 @@
 // aggregates and that kernels must read those counts rather than size work
 // from buffer capacities.
 //
-// Three kernels, no inter-block waiting:
-//   1. count:  one block per tile of LAYOUT_TILE tokens builds the tile's
-//              per-expert histogram in shared memory, writes in_rank for its
-//              tokens and the tile's per-rank token counts.
-//   2. scan:   one warp per expert column turns the tile histograms into
-//              exclusive per-tile offsets (in place) and the expert totals;
-//              extra warps total the per-rank token counts.
-//   3. slot:   one block per tile scans the expert totals, then each warp
-//              orders its share of the tile's (t, j) pairs with match_any so
-//              that rows inside an expert follow (t, j) order.
+// Kernels (no block ever waits for another block):
+//   count:  one block per tile of tokens builds the tile's per-expert
+//           histogram in shared memory, writes in_rank for its tokens, the
+//           tile's per-rank token counts and the tile's status bits.
+//   [scan]: only for more than LAYOUT_FUSED_MAX_TILES tiles: one warp per
+//           expert column turns the tile histograms into exclusive per-tile
+//           offsets (in place) and the expert totals.
+//   slot:   one block per tile.  With few tiles it first sums, for every
+//           expert, the histograms of the tiles before it and of all tiles;
+//           then it scans the expert totals, and each warp orders its share
+//           of the tile's (t, j) pairs with match_any so that rows inside an
+//           expert follow (t, j) order.
 // Shared-memory atomics only count; no order is decided by an atomic.
 #include "ep_device.cuh"
 #include "ep_internal.h"
@@ -55,16 +57,20 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_count_kernel(LayoutArgs
     extern __shared__ int smem[];
     int *hist = smem;          // [P]
     int *tokr = hist + a.P;    // [R]
-    int *pp = tokr + a.R;      // [LAYOUT_TILE * k]
+    int *pp = tokr + a.R;      // [tile_tokens * k]
+    __shared__ int bad_sh;
 
+    pdl_launch_dependents();
     const int tile = blockIdx.x;
-    const int t0 = tile * LAYOUT_TILE;
-    const int nt = min(LAYOUT_TILE, a.T - t0);
+    const int t0 = tile * a.tile_tokens;
+    const int nt = min(a.tile_tokens, a.T - t0);
     const int npairs = nt * a.k;
 
     for (int i = threadIdx.x; i < a.P; i += blockDim.x) hist[i] = 0;
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) tokr[i] = 0;
+    if (threadIdx.x == 0) bad_sh = 0;
     __syncthreads();
+    pdl_wait();
 
     int bad = 0;
     for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_count_kernel(LayoutArgs
         pp[i] = p;
         if (p >= 0) atomicAdd(&hist[p], 1);
     }
-    if (bad && a.dev_status != nullptr) atomicOr(a.dev_status, bad);
+    if (bad) atomicOr(&bad_sh, bad);
     __syncthreads();
 
     const int epr = a.P / a.R;
@@ -90,11 +96,15 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_count_kernel(LayoutArgs
 
     for (int i = threadIdx.x; i < a.P; i += blockDim.x) a.tile_cnt[(size_t)tile * a.P + i] = hist[i];
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) a.tile_tok[(size_t)tile * a.R + i] = tokr[i];
+    if (threadIdx.x == 0) a.tile_bad[tile] = bad_sh;
 }
 
-// warp per column: columns [0, P) are experts, [P, P+R) are ranks
-__global__ void __launch_bounds__(LAYOUT_THREADS) layout_scan_kernel(LayoutArgs a, int NT)
+// many tiles: warp per column, columns [0, P) are experts, [P, P+R) ranks
+__global__ void __launch_bounds__(LAYOUT_THREADS) layout_scan_kernel(LayoutArgs a)
 {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int NT = a.n_tiles;
     const int lane = threadIdx.x & 31;
     const int col = blockIdx.x * LAYOUT_WARPS + (threadIdx.x >> 5);
     if (col >= a.P + a.R) return;  // warp-uniform
@@ -148,26 +158,80 @@ __device__ int block_exclusive_scan(int *v, int n, int *warp_tot)
     return total;
 }
 
+template <bool FUSED>
 __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs a)
 {
     extern __shared__ int smem[];
-    int *eoff = smem;                          // [P + 1]
-    int *whist = eoff + a.P + 1;               // [LAYOUT_WARPS][P]
-    int *pp = whist + LAYOUT_WARPS * a.P;      // [LAYOUT_TILE * k]
+    int *eoff = smem;                          // [P + 1]  expert start rows
+    int *toff = eoff + a.P + 1;                // [P]      rows of earlier tiles
+    int *whist = toff + a.P;                   // [LAYOUT_WARPS][P]
+    int *pp = whist + LAYOUT_WARPS * a.P;      // [tile_tokens * k]
     __shared__ int warp_tot[LAYOUT_WARPS + 1];
 
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int tile = blockIdx.x;
-    const int t0 = tile * LAYOUT_TILE;
-    const int nt = min(LAYOUT_TILE, a.T - t0);
+    const int NT = a.n_tiles;
+    const int t0 = tile * a.tile_tokens;
+    const int nt = min(a.tile_tokens, a.T - t0);
     const int npairs = nt * a.k;
-
-    for (int i = threadIdx.x; i < a.P; i += blockDim.x) eoff[i] = a.cnt_expert[i];
     for (int i = threadIdx.x; i < LAYOUT_WARPS * a.P; i += blockDim.x) whist[i] = 0;
-    int bad = 0;  // already reported by the count kernel
+    pdl_wait();
+
+    if (FUSED) {
+        // per expert: rows in tiles before this one, and in all tiles; eight
+        // independent loads in flight per thread (the column is in L2)
+        for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
+            int before = 0, total = 0;
+            for (int i0 = 0; i0 < NT; i0 += 8) {
+                int c[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    c[u] = (i0 + u < NT) ? __ldg(a.tile_cnt + (size_t)(i0 + u) * a.P + p) : 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    before += (i0 + u < tile) ? c[u] : 0;
+                    total += c[u];
+                }
+            }
+            toff[p] = before;
+            eoff[p] = total;
+        }
+    } else {
+        for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
+            toff[p] = a.tile_cnt[(size_t)tile * a.P + p];  // exclusive, from the scan
+            eoff[p] = a.cnt_expert[p];
+        }
+    }
+    int bad = 0;  // reported below from the count kernel's tile status words
     for (int i = threadIdx.x; i < npairs; i += blockDim.x)
         pp[i] = phys_expert(a, t0 + i / a.k, i % a.k, bad);
     __syncthreads();
+
+    if (tile == 0) {
+        if (FUSED) {
+            for (int p = threadIdx.x; p < a.P; p += blockDim.x) a.cnt_expert[p] = eoff[p];
+            for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+                int sum = 0;
+                for (int i0 = 0; i0 < NT; i0 += 8) {
+                    int c[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        c[u] = (i0 + u < NT) ? __ldg(a.tile_tok + (size_t)(i0 + u) * a.R + r) : 0;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) sum += c[u];
+                }
+                a.tok_rank[r] = sum;
+            }
+        }
+        if (a.dev_status != nullptr && threadIdx.x < 32) {
+            int st = 0;
+            for (int i = threadIdx.x; i < NT; i += 32) st |= a.tile_bad[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) st |= __shfl_xor_sync(FULL_MASK, st, off);
+            if (threadIdx.x == 0) *a.dev_status = st;
+        }
+    }
     const int total = block_exclusive_scan(eoff, a.P, warp_tot);
     if (threadIdx.x == 0) eoff[a.P] = total;
     __syncthreads();
@@ -191,10 +255,10 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
         if (p >= 0) atomicAdd(&my[p], 1);
     }
     __syncthreads();
-    // per expert: base row of each warp's share = expert start + tile offset
-    // + rows of earlier warps in this tile
+    // per expert: first row of each warp's share = expert start + rows of
+    // earlier tiles + rows of earlier warps in this tile
     for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
-        int base = eoff[p] + a.tile_cnt[(size_t)tile * a.P + p];
+        int base = eoff[p] + toff[p];
 #pragma unroll
         for (int w = 0; w < LAYOUT_WARPS; ++w) {
             const int c = whist[w * a.P + p];
@@ -228,6 +292,8 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
 
 __global__ void layout_empty_kernel(LayoutArgs a)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     for (int i = threadIdx.x; i < a.P; i += blockDim.x) a.cnt_expert[i] = 0;
     for (int i = threadIdx.x; i <= a.P; i += blockDim.x) a.expert_off[i] = 0;
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) {
@@ -235,6 +301,13 @@ __global__ void layout_empty_kernel(LayoutArgs a)
         a.tok_rank[i] = 0;
     }
     for (int i = threadIdx.x; i <= a.R; i += blockDim.x) a.rank_off[i] = 0;
+    if (threadIdx.x == 0 && a.dev_status != nullptr) *a.dev_status = 0;
+}
+
+void opt_in_smem(const void *fn, size_t bytes)
+{
+    if (bytes > 48 * 1024)
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 }  // namespace
@@ -242,37 +315,24 @@ __global__ void layout_empty_kernel(LayoutArgs a)
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
 {
     cudaError_t err;
-    if (a.dev_status != nullptr) {
-        err = cudaMemsetAsync(a.dev_status, 0, sizeof(int32_t), s);
-        if (err != cudaSuccess) return err;
-    }
-    if (a.T == 0) {
-        layout_empty_kernel<<<1, 256, 0, s>>>(a);
-        return cudaGetLastError();
-    }
-    const int NT = layout_tiles(a.T);
-    const size_t sm_count = sizeof(int) * ((size_t)a.P + a.R + (size_t)LAYOUT_TILE * a.k);
+    if (a.T == 0) return launch_pdl(layout_empty_kernel, dim3(1), dim3(256), 0, s, a);
+    const int NT = a.n_tiles;
+    const size_t pairs = (size_t)a.tile_tokens * a.k;
+    const size_t sm_count = sizeof(int) * ((size_t)a.P + a.R + pairs);
     const size_t sm_slot =
-        sizeof(int) * ((size_t)a.P + 1 + (size_t)LAYOUT_WARPS * a.P + (size_t)LAYOUT_TILE * a.k);
-    if (sm_slot > 48 * 1024 || sm_count > 48 * 1024) {  // opt in above 48 KB
-        static volatile int attr_set[64] = {0};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 64 || !attr_set[dev]) {
-            cudaFuncSetAttribute(layout_count_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            cudaFuncSetAttribute(layout_slot_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            if (dev < 64) attr_set[dev] = 1;
-        }
-    }
-    layout_count_kernel<<<NT, LAYOUT_THREADS, sm_count, s>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        sizeof(int) * ((size_t)2 * a.P + 1 + (size_t)LAYOUT_WARPS * a.P + pairs);
+    const bool fused = NT <= LAYOUT_FUSED_MAX_TILES;
+    opt_in_smem((const void *)layout_count_kernel, sm_count);
+    opt_in_smem(fused ? (const void *)layout_slot_kernel<true> : (const void *)layout_slot_kernel<false>,
+                sm_slot);
+    err = launch_pdl(layout_count_kernel, dim3(NT), dim3(LAYOUT_THREADS), sm_count, s, a);
+    if (err != cudaSuccess) return err;
+    if (fused) return launch_pdl(layout_slot_kernel<true>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
     const int cols = a.P + a.R;
-    layout_scan_kernel<<<(cols + LAYOUT_WARPS - 1) / LAYOUT_WARPS, LAYOUT_THREADS, 0, s>>>(a, NT);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    layout_slot_kernel<<<NT, LAYOUT_THREADS, sm_slot, s>>>(a);
-    return cudaGetLastError();
+    err = launch_pdl(layout_scan_kernel, dim3((cols + LAYOUT_WARPS - 1) / LAYOUT_WARPS),
+                     dim3(LAYOUT_THREADS), 0, s, a);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(layout_slot_kernel<false>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
 }
 
 }  // namespace ep

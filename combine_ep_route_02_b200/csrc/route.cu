@@ -47,6 +47,7 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
              int G, int Kg, int k, float scale, int renorm, int vec4,
              int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
 {
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
     const int e0 = lane * EPL;
@@ -58,6 +59,7 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
     const int lanes_per_group = aligned ? lpg : 0;
     const int my_group = (e0 < E) ? e0 / gs : -1;        // valid when aligned
 
+    pdl_wait();
     float b[EPL];
     int gid[EPL];  // token-invariant group of each held expert (-1: none)
 #pragma unroll
@@ -228,9 +230,9 @@ cudaError_t launch_epl(const RouteArgs &a, int vec4, cudaStream_t s)
     int blocks = (a.T + warps_per_block - 1) / warps_per_block;
     const int cap = device_sm_count() * 16;
     if (blocks > cap) blocks = cap;
-    route_kernel<EPL><<<blocks, warps_per_block * 32, 0, s>>>(
-        a.logits, a.bias, a.T, a.E, a.G, a.Kg, a.k, a.scale, a.renorm, vec4, a.topk_idx, a.topk_w);
-    return cudaGetLastError();
+    return launch_pdl(route_kernel<EPL>, dim3(blocks), dim3(warps_per_block * 32), 0, s, a.logits,
+                      a.bias, a.T, a.E, a.G, a.Kg, a.k, a.scale, a.renorm, vec4, a.topk_idx,
+                      a.topk_w);
 }
 
 }  // namespace

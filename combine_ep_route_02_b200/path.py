@@ -56,7 +56,8 @@ class EpPath:
         self.in_rank = torch.empty((T, R), device=dev, dtype=torch.uint8)
         self.slot = torch.empty((T, k), **i32)
         self.src = torch.empty(T * k, **i32)
-        self.dev_status = torch.zeros(1, **i32)
+        self.dev_status = torch.zeros(1, **i32)    # layout (cleared by each layout call)
+        self.copy_status = torch.zeros(1, **i32)   # dispatch / combine (sticky)
         ws = B.ep_workspace_size(T, k, P, R)
         self.workspace = torch.empty(max(ws, 256), device=dev, dtype=torch.uint8)
         if self.fp8:
@@ -80,11 +81,11 @@ class EpPath:
 
     def dispatch(self, x: torch.Tensor, stream=None):
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
-                      self.recv_scale, self.num_sms, stream)
+                      self.recv_scale, self.num_sms, self.copy_status, stream)
 
     def combine(self, y: torch.Tensor, stream=None):
         B.ep_combine(y, self.slot, self.topk_w, self.T, self.H, self.k, self.out,
-                     self.num_sms, stream)
+                     self.num_sms, self.copy_status, stream)
 
     def step(self, x, logits, bias, y, stream=None):
         """route, layout, dispatch, then combine of the expert outputs y."""
@@ -95,12 +96,22 @@ class EpPath:
         return self.out
 
     def kernels_per_step(self) -> int:
-        # route 1, layout 3 (+1 memset node), dispatch 1, combine 1
-        return 6 if self.T > 0 else 1
+        """Kernels one step launches: route, layout (count + slot, plus a
+        column scan above 64 tiles), dispatch, combine.  Mirrors the tiling
+        rule of the layout (64..512 tokens per tile, at most 64 tiles while
+        tiles can grow, capped by the slot kernel's shared memory)."""
+        if self.T == 0:
+            return 1
+        tt = max(64, min(512, -(-self.T // 64)))
+        cap = max(32, ((51200 - 10 * self.P - 1) // self.k) // 32 * 32)
+        tt = min(tt, cap)
+        n_tiles = -(-self.T // tt)
+        return 1 + (2 if n_tiles <= 64 else 3) + 1 + 1
 
     def check_status(self):
-        """Reads the device status word (synchronises); raises on bad data."""
-        st = int(self.dev_status.item())
+        """Reads the device status words (synchronises); raises on bad data
+        or a timed-out copy."""
+        st = int(self.dev_status.item()) | int(self.copy_status.item())
         if st:
-            raise B.EpError("ep_dispatch_layout", B.EP_ERR_DEVICE)
+            raise B.EpError("ep path (device status %#x)" % st, B.EP_ERR_DEVICE)
         return st

@@ -67,9 +67,11 @@ typedef enum {
     EP_ERR_DEVICE = 4       /* reserved for callers mapping *dev_status */
 } ep_status;
 
-/* Bits written to *dev_status by ep_dispatch_layout. */
-#define EP_DEV_BAD_EXPERT 1  /* a topk_idx entry outside [0, E) */
-#define EP_DEV_BAD_REPLICA 2 /* n_rep[e] outside [1, max_rep] or phys id outside [0, P) */
+/* Bits reported through a caller's *dev_status word. */
+#define EP_DEV_BAD_EXPERT 1  /* layout: a topk_idx entry outside [0, E) */
+#define EP_DEV_BAD_REPLICA 2 /* layout: n_rep[e] outside [1, max_rep] or phys id outside [0, P) */
+#define EP_DEV_TIMEOUT 4     /* dispatch / combine: a bounded wait for an asynchronous copy
+                                gave up; that call's output is incomplete */
 
 /* Same object as cudaStream_t; no CUDA header is needed to use this API. */
 typedef struct CUstream_st *ep_stream_t;
@@ -163,12 +165,17 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
  *               fp32(amax / 448), q = e4m3_rn_satfinite(fp32(x / scale));
  *               a block with amax == 0 gets scale 0 and zero bytes
  *   num_sms     SMs to spread the work over (0 = all), like DeepEP's num_sms
+ *   dev_status  int32 [1] or NULL: EP_DEV_TIMEOUT is ORed in if a bounded
+ *               wait on a TMA copy gives up (the word is not cleared here)
  *
  * Slots outside [0, T*k) are skipped (rows they would fill are left as they
- * were).  recv_x must be 16-byte aligned, recv_scale 4-byte aligned.
+ * were).  recv_x must be 16-byte aligned, recv_scale 4-byte aligned.  With
+ * fp8, H % 512 == 0 and a 16-byte aligned recv_scale, rows move through
+ * shared memory by TMA bulk copies; otherwise by 16-byte thread stores.
  */
 ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
-                      void *recv_x, float *recv_scale, int num_sms, ep_stream_t stream);
+                      void *recv_x, float *recv_scale, int num_sms, int32_t *dev_status,
+                      ep_stream_t stream);
 
 /*
  * Combine: weighted gather-reduce back to token order.
@@ -180,9 +187,11 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *sl
  * out[t] = bf16_rne( acc ), acc = fp32 sum over j = 0..k-1 in order of
  * fp32(w[t,j] * y[slot[t,j]]), each step rounded to nearest even.  Slots
  * outside [0, T*k) contribute nothing.  y and out 16-byte aligned, H % 8 == 0.
+ * dev_status as for ep_dispatch (NULL allowed).
  */
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T,
-                     int H, int k, void *out_bf16, int num_sms, ep_stream_t stream);
+                     int H, int k, void *out_bf16, int num_sms, int32_t *dev_status,
+                     ep_stream_t stream);
 
 /*
  * Allocation-free variant of ep_dispatch_layout.  It has no counterpart in
@@ -197,7 +206,7 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
  * EP_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
  * the library keeps until the process exits.  Sizes whose
  * ep_workspace_size(T, k, P, R) exceeds that limit return
- * EP_ERR_UNSUPPORTED (with P = 256 and R = 8 that is about 250K tokens).
+ * EP_ERR_UNSUPPORTED (with k = 8, P = 256 and R = 8 that is about 2M tokens).
  * The first call on each device looks up the array's device address (host
  * code cannot use the array's name as a device pointer); make that first
  * call before any stream capture.  The call allocates and frees nothing.

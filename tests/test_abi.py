@@ -42,9 +42,11 @@ def test_status_strings(lib):
 
 
 def test_workspace_size(lib):
-    # 64-token tiles; [NT][P] + [NT][R] int32, each rounded to 256 bytes
-    assert ep.ep_workspace_size(8192, 8, 256, 8) == 128 * 256 * 4 + 4096
-    assert ep.ep_workspace_size(1, 8, 288, 32) == 1280 + 256
+    # NT tiles of max(64, ceil(T/64)) tokens; [NT][P] + [NT][R] + [NT] int32,
+    # each rounded up to 256 bytes
+    assert ep.ep_workspace_size(8192, 8, 256, 8) == 64 * 256 * 4 + 2048 + 256
+    assert ep.ep_workspace_size(1, 8, 288, 32) == 1280 + 256 + 256
+    assert ep.ep_workspace_size(16384, 8, 288, 32) == 64 * 288 * 4 + 64 * 32 * 4 + 256
     assert ep.ep_workspace_size(0, 8, 256, 8) > 0
     assert ep.ep_workspace_size(-1, 8, 256, 8) == 0
     assert ep.ep_workspace_size(10, 0, 256, 8) == 0
@@ -101,7 +103,7 @@ def test_layout_rejects_too_many_experts(lib):
     (FAKE, 4, 256, 0, FAKE, 1, FAKE, FAKE),
 ])
 def test_dispatch_rejects_invalid(lib, args):
-    assert lib.ep_dispatch(*args, 0, None) == B.EP_ERR_INVALID
+    assert lib.ep_dispatch(*args, 0, None, None) == B.EP_ERR_INVALID
 
 
 @pytest.mark.parametrize("args", [
@@ -111,7 +113,7 @@ def test_dispatch_rejects_invalid(lib, args):
     (FAKE, FAKE, FAKE, -1, 256, 2, FAKE),
 ])
 def test_combine_rejects_invalid(lib, args):
-    assert lib.ep_combine(*args, 0, None) == B.EP_ERR_INVALID
+    assert lib.ep_combine(*args, 0, None, None) == B.EP_ERR_INVALID
 
 
 def test_binding_raises(lib):

@@ -128,7 +128,7 @@ def test_layout_full_size(name):
         assert np.array_equal(got[n].reshape(ref[n].shape), ref[n]), n
 
 
-@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 1000, 4097])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 1000, 4097, 40000])
 @pytest.mark.parametrize("name", ["ds16b", "skew"])
 def test_layout_ragged(T, name):
     cfg = CONFIGS[name].scaled(T)
@@ -152,12 +152,15 @@ def test_layout_empty():
         assert (getattr(path, n) == 0).all(), n
 
 
-def test_layout_max_sizes_and_skewed_ids():
-    """P = 4096 physical experts, k = 32, R = 64, heavily skewed expert ids"""
+@pytest.mark.parametrize("T", [700, 20000])
+def test_layout_max_sizes_and_skewed_ids(T):
+    """P = 4096 physical experts, k = 32, R = 64, heavily skewed expert ids;
+    T = 20000 takes more tiles than the slot kernel sums itself, with the
+    largest tiles its shared memory allows"""
     from combine_ep_route_02_b200 import ep_dispatch_layout, ep_workspace_size
     rng = np.random.default_rng(11)
-    T, k, E, R = 700, 32, 4096, 64
-    idx = np.stack([rng.choice(E, k, replace=False, p=None) for _ in range(T)]).astype(np.int32)
+    k, E, R = 32, 4096, 64
+    idx = np.argsort(rng.random((T, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
     idx[::3, :8] = np.arange(8)  # many tokens on the same few experts
     ref = oracle.layout(idx, E, E, R)
     d = dict(cnt_expert=E, expert_off=E + 1, rows_rank=R, rank_off=R + 1, tok_rank=R,
@@ -306,6 +309,26 @@ def test_dispatch_num_sms_and_invalid_slots(num_sms):
     assert np.array_equal(got[written], rx[written])
     assert np.array_equal(gs[written], rs[written])
     assert (got[unwritten] == 0xAB).all() and (gs[unwritten] == -1.0).all()
+
+
+def test_dispatch_fp8_thread_store_path():
+    """a recv_scale that is 4- but not 16-byte aligned takes the thread-store
+    kernel instead of the TMA pipeline; both must give the oracle's bytes"""
+    cfg = CONFIGS["v3"].scaled(300)
+    wl = Workload(cfg, seed=6)
+    idx, _, _ = oracle_route(cfg, wl)
+    lay = oracle_layout(cfg, wl, idx)
+    from combine_ep_route_02_b200 import ep_dispatch
+    T, H, k = cfg.T, cfg.H, cfg.topk
+    rx = torch.empty((T * k, H), dtype=torch.uint8, device="cuda")
+    rs_buf = torch.empty(T * k * (H // 128) + 1, dtype=torch.float32, device="cuda")
+    rs = rs_buf[1:].view(T * k, H // 128)
+    assert rs.data_ptr() % 16 == 4
+    ep_dispatch(wl.x.cuda(), T, H, k, torch.from_numpy(lay["slot"]).cuda(), True, rx, rs)
+    torch.cuda.synchronize()
+    ref_x, ref_s = oracle.dispatch(wl.x, lay["slot"], True)
+    assert np.array_equal(rx.cpu().numpy(), ref_x)
+    assert np.array_equal(rs.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
 
 
 def test_dispatch_bf16_ragged():

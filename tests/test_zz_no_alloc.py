@@ -86,7 +86,7 @@ def test_noalloc_layout_matches_workspace_layout_twice():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     P, R, k = 256, 8, 8
-    T = 300000  # needs more than the 4 MiB of fixed scratch
+    T = 3000000  # needs more than the 4 MiB of fixed scratch
     assert B.ep_workspace_size(T, k, P, R) > 4 << 20
     st = B.lib().ep_dispatch_layout_noalloc(None, T, k, P, P, R, None, None, 0, *([None] * 8),
                                             None, None)
