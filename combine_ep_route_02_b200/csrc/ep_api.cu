@@ -127,7 +127,7 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
     LayoutArgs a{topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
                  cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
                  reinterpret_cast<int32_t *>(ws), reinterpret_cast<int32_t *>(ws + o1),
-                 reinterpret_cast<int32_t *>(ws + o2), dev_status, layout_tile_tokens(T, k, P), NT};
+                 reinterpret_cast<int32_t *>(ws + o2), dev_status, layout_tile_tokens(T, k, P), NT, layout_hist_warps(P)};
     return from_cuda(launch_layout(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

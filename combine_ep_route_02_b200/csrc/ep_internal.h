@@ -14,7 +14,7 @@ namespace ep {
 constexpr int LAYOUT_MIN_TILE = 64;
 constexpr int LAYOUT_MAX_TILE = 512;
 constexpr int LAYOUT_FUSED_MAX_TILES = 64;
-constexpr int LAYOUT_THREADS = 256;
+constexpr int LAYOUT_THREADS = 1024;
 constexpr int LAYOUT_WARPS = LAYOUT_THREADS / 32;
 constexpr int MAX_EXPERTS = 1024;   // logical experts (routing)
 constexpr int MAX_PHYS = 4096;      // physical experts (layout)
@@ -46,6 +46,7 @@ struct LayoutArgs {
     int32_t *dev_status;
     int tile_tokens;    // TT
     int n_tiles;        // NT
+    int hist_warps;     // slot-kernel warps that order pairs
 };
 
 struct DispatchArgs {
@@ -69,16 +70,26 @@ struct CombineArgs {
     int grid;
 };
 
+// Warps of the slot kernel that each order one contiguous share of a tile's
+// pairs (each keeps a P-entry table in shared memory): 32, or fewer for
+// large P so that the tables stay within 128 KB.
+inline int layout_hist_warps(int P)
+{
+    int w = LAYOUT_WARPS;
+    while (w > 1 && (size_t)w * P > 32768) w >>= 1;
+    return w;
+}
+
 // Tokens per tile: enough for at most LAYOUT_FUSED_MAX_TILES tiles, within
 // [LAYOUT_MIN_TILE, LAYOUT_MAX_TILE], and small enough that the slot kernel's
-// shared memory ((10 P + 1) ints of tables + tile_tokens * k ints of pair
-// ids) stays under 200 KB.
+// shared memory ((2 P + 1) + hist_warps * P ints of tables + tile_tokens * k
+// ints of pair ids) stays under 200 KB.
 inline int layout_tile_tokens(int T, int k, int P)
 {
     int tt = (T + LAYOUT_FUSED_MAX_TILES - 1) / LAYOUT_FUSED_MAX_TILES;
     if (tt < LAYOUT_MIN_TILE) tt = LAYOUT_MIN_TILE;
     if (tt > LAYOUT_MAX_TILE) tt = LAYOUT_MAX_TILE;
-    int cap = (51200 - 10 * P - 1) / (k > 0 ? k : 1);
+    int cap = (51200 - (2 * P + 1) - layout_hist_warps(P) * P) / (k > 0 ? k : 1);
     cap = (cap / 32) * 32;
     if (cap < 32) cap = 32;
     return tt < cap ? tt : cap;

@@ -99,14 +99,17 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_count_kernel(LayoutArgs
     if (threadIdx.x == 0) a.tile_bad[tile] = bad_sh;
 }
 
+constexpr int SCAN_THREADS = 256;
+constexpr int SCAN_WARPS = SCAN_THREADS / 32;
+
 // many tiles: warp per column, columns [0, P) are experts, [P, P+R) ranks
-__global__ void __launch_bounds__(LAYOUT_THREADS) layout_scan_kernel(LayoutArgs a)
+__global__ void __launch_bounds__(SCAN_THREADS) layout_scan_kernel(LayoutArgs a)
 {
     pdl_launch_dependents();
     pdl_wait();
     const int NT = a.n_tiles;
     const int lane = threadIdx.x & 31;
-    const int col = blockIdx.x * LAYOUT_WARPS + (threadIdx.x >> 5);
+    const int col = blockIdx.x * SCAN_WARPS + (threadIdx.x >> 5);
     if (col >= a.P + a.R) return;  // warp-uniform
     if (col < a.P) {
         int running = 0;
@@ -162,10 +165,11 @@ template <bool FUSED>
 __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs a)
 {
     extern __shared__ int smem[];
+    const int HW = a.hist_warps;
     int *eoff = smem;                          // [P + 1]  expert start rows
     int *toff = eoff + a.P + 1;                // [P]      rows of earlier tiles
-    int *whist = toff + a.P;                   // [LAYOUT_WARPS][P]
-    int *pp = whist + LAYOUT_WARPS * a.P;      // [tile_tokens * k]
+    int *whist = toff + a.P;                   // [HW][P]
+    int *pp = whist + HW * a.P;                // [tile_tokens * k]
     __shared__ int warp_tot[LAYOUT_WARPS + 1];
 
     pdl_launch_dependents();
@@ -175,27 +179,42 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
     const int t0 = tile * a.tile_tokens;
     const int nt = min(a.tile_tokens, a.T - t0);
     const int npairs = nt * a.k;
-    for (int i = threadIdx.x; i < LAYOUT_WARPS * a.P; i += blockDim.x) whist[i] = 0;
+    for (int i = threadIdx.x; i < HW * a.P; i += blockDim.x) whist[i] = 0;
     pdl_wait();
 
     if (FUSED) {
-        // per expert: rows in tiles before this one, and in all tiles; eight
-        // independent loads in flight per thread (the column is in L2)
-        for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
+        // per expert: rows in tiles before this one, and in all tiles.  Four
+        // consecutive lanes share a column, each summing every fourth tile
+        // with four loads in flight, then combine by shuffles.
+        constexpr int PARTS = 4;
+        for (int base = 0; base < a.P; base += LAYOUT_THREADS / PARTS) {
+            const int p = base + (int)threadIdx.x / PARTS;
+            const int part = threadIdx.x % PARTS;
             int before = 0, total = 0;
-            for (int i0 = 0; i0 < NT; i0 += 8) {
-                int c[8];
+            if (p < a.P) {
+                for (int i0 = part; i0 < NT; i0 += 4 * PARTS) {
+                    int c[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    c[u] = (i0 + u < NT) ? __ldg(a.tile_cnt + (size_t)(i0 + u) * a.P + p) : 0;
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * PARTS;
+                        c[u] = (i < NT) ? __ldg(a.tile_cnt + (size_t)i * a.P + p) : 0;
+                    }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    before += (i0 + u < tile) ? c[u] : 0;
-                    total += c[u];
+                    for (int u = 0; u < 4; ++u) {
+                        before += (i0 + u * PARTS < tile) ? c[u] : 0;
+                        total += c[u];
+                    }
                 }
             }
-            toff[p] = before;
-            eoff[p] = total;
+#pragma unroll
+            for (int off = 1; off < PARTS; off <<= 1) {
+                before += __shfl_xor_sync(FULL_MASK, before, off);
+                total += __shfl_xor_sync(FULL_MASK, total, off);
+            }
+            if (part == 0 && p < a.P) {
+                toff[p] = before;
+                eoff[p] = total;
+            }
         }
     } else {
         for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
@@ -246,21 +265,22 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
         if (threadIdx.x == 0) a.rank_off[a.R] = total;
     }
 
-    // each warp owns a contiguous share of the tile's pairs, in (t, j) order
-    const int per = (npairs + LAYOUT_WARPS - 1) / LAYOUT_WARPS;
-    const int lo = min(npairs, warp * per), hi = min(npairs, lo + per);
-    int *my = whist + warp * a.P;
+    // warps w < HW each own a contiguous share of the tile's pairs, in (t, j)
+    // order (warps w >= HW get an empty share)
+    const int per = (npairs + HW - 1) / HW;
+    const int lo = warp < HW ? min(npairs, warp * per) : npairs;
+    const int hi = warp < HW ? min(npairs, lo + per) : npairs;
+    int *my = whist + (warp < HW ? warp : 0) * a.P;
     for (int i = lo + lane; i < hi; i += 32) {
         const int p = pp[i];
         if (p >= 0) atomicAdd(&my[p], 1);
     }
     __syncthreads();
-    // per expert: first row of each warp's share = expert start + rows of
-    // earlier tiles + rows of earlier warps in this tile
+    // per expert: first row of each share = expert start + rows of earlier
+    // tiles + rows of earlier shares in this tile
     for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
         int base = eoff[p] + toff[p];
-#pragma unroll
-        for (int w = 0; w < LAYOUT_WARPS; ++w) {
+        for (int w = 0; w < HW; ++w) {
             const int c = whist[w * a.P + p];
             whist[w * a.P + p] = base;
             base += c;
@@ -320,7 +340,7 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
     const size_t pairs = (size_t)a.tile_tokens * a.k;
     const size_t sm_count = sizeof(int) * ((size_t)a.P + a.R + pairs);
     const size_t sm_slot =
-        sizeof(int) * ((size_t)2 * a.P + 1 + (size_t)LAYOUT_WARPS * a.P + pairs);
+        sizeof(int) * ((size_t)2 * a.P + 1 + (size_t)a.hist_warps * a.P + pairs);
     const bool fused = NT <= LAYOUT_FUSED_MAX_TILES;
     opt_in_smem((const void *)layout_count_kernel, sm_count);
     opt_in_smem(fused ? (const void *)layout_slot_kernel<true> : (const void *)layout_slot_kernel<false>,
@@ -329,8 +349,8 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
     if (err != cudaSuccess) return err;
     if (fused) return launch_pdl(layout_slot_kernel<true>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
     const int cols = a.P + a.R;
-    err = launch_pdl(layout_scan_kernel, dim3((cols + LAYOUT_WARPS - 1) / LAYOUT_WARPS),
-                     dim3(LAYOUT_THREADS), 0, s, a);
+    err = launch_pdl(layout_scan_kernel, dim3((cols + SCAN_WARPS - 1) / SCAN_WARPS),
+                     dim3(SCAN_THREADS), 0, s, a);
     if (err != cudaSuccess) return err;
     return launch_pdl(layout_slot_kernel<false>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
 }

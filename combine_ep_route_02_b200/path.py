@@ -103,7 +103,10 @@ class EpPath:
         if self.T == 0:
             return 1
         tt = max(64, min(512, -(-self.T // 64)))
-        cap = max(32, ((51200 - 10 * self.P - 1) // self.k) // 32 * 32)
+        hw = 32
+        while hw > 1 and hw * self.P > 32768:
+            hw //= 2
+        cap = max(32, ((51200 - (2 * self.P + 1) - hw * self.P) // self.k) // 32 * 32)
         tt = min(tt, cap)
         n_tiles = -(-self.T // tt)
         return 1 + (2 if n_tiles <= 64 else 3) + 1 + 1
