@@ -88,6 +88,31 @@ def test_route_shapes(E, G, Kg, k, kind):
         assert np.array_equal(gwn[ok].view(np.uint32), w[ok].view(np.uint32))
 
 
+def test_route_sigmoid_every_expert():
+    """one group, k = E, no renorm, scale 1: the weights are the fp32
+    sigmoids themselves, so every one is compared with the oracle's fp64
+    evaluation (saturation, underflow and infinities included)"""
+    from combine_ep_route_02_b200 import RouteCfg, ep_route
+    rng = np.random.default_rng(21)
+    E, T = 32, 65536
+    edges = np.array([0.0, -0.0, 1e-30, -1e-30, 17.0, 17.33, -17.0, 88.0, -88.0, -87.3,
+                      -103.28, -103.3, -103.97, -104.0, -110.0, 700.0, -700.0, 701.0,
+                      -701.0, 1e30, -1e30, np.inf, -np.inf], np.float32)
+    logits = np.concatenate([
+        rng.normal(0, 1, T * E // 2), rng.normal(0, 8, T * E // 4),
+        rng.uniform(-110, 110, T * E // 4 - edges.size)]).astype(np.float32)
+    logits = np.concatenate([logits, edges]).reshape(T, E)
+    cfg = RouteCfg(E, 1, 1, E, 1.0, 0)
+    gidx = torch.empty((T, E), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    ep_route(torch.from_numpy(logits).cuda(), None, T, cfg, gidx, gw)
+    idx, w, hard = oracle.route(logits, None, 1, 1, E, 1.0, False)
+    ok = hard == 0
+    assert np.array_equal(gidx.cpu().numpy()[ok], idx[ok])
+    assert np.array_equal(gw.cpu().numpy()[ok].view(np.uint32), w[ok].view(np.uint32))
+    assert (~ok).sum() <= 2
+
+
 def test_route_empty_and_single():
     from combine_ep_route_02_b200 import RouteCfg, ep_route
     cfg = RouteCfg(256, 8, 4, 8, 2.5, 1)
