@@ -109,7 +109,7 @@ EP_DEV int warp_pick(uint32_t key, int idx)
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, EPL <= 8 ? 4 : 1)
 route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int T, int E,
              int G, int Kg, int k, float scale, int renorm, int vec4,
              int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
@@ -238,9 +238,16 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
                     chosen |= 1u << g;
                 }
             }
+            if (aligned) {
+                // the lane's experts share one group
+                if (my_group >= 0 && !((chosen >> my_group) & 1u))
 #pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) key[i] = NONE;
+                    for (int i = 0; i < EPL; ++i) key[i] = NONE;
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) key[i] = NONE;
+            }
         }
 
         // lane-local best: the first (lowest index) of the largest keys;
@@ -300,9 +307,21 @@ route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, i
 template <int EPL>
 cudaError_t launch_epl(const RouteArgs &a, int vec4, cudaStream_t s)
 {
+    // persistent warps: one wave of resident blocks, each warp looping over
+    // tokens, so no partly filled last wave
     const int warps_per_block = 8;
     int blocks = (a.T + warps_per_block - 1) / warps_per_block;
-    const int cap = device_sm_count() * 16;
+    static volatile int occ[64][6] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int slot = EPL == 1 ? 0 : EPL == 2 ? 1 : EPL == 4 ? 2 : EPL == 8 ? 3 : EPL == 16 ? 4 : 5;
+    int per_sm = dev < 64 ? occ[dev][slot] : 0;
+    if (per_sm <= 0) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_kernel<EPL>, 256, 0);
+        if (per_sm <= 0) per_sm = 1;
+        if (dev < 64) occ[dev][slot] = per_sm;
+    }
+    const int cap = device_sm_count() * per_sm;
     if (blocks > cap) blocks = cap;
     return launch_pdl(route_kernel<EPL>, dim3(blocks), dim3(warps_per_block * 32), 0, s, a.logits,
                       a.bias, a.T, a.E, a.G, a.Kg, a.k, a.scale, a.renorm, vec4, a.topk_idx,

@@ -83,17 +83,18 @@ class EpPath:
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
                       self.recv_scale, self.num_sms, self.copy_status, stream)
 
-    def combine(self, y: torch.Tensor, stream=None):
-        B.ep_combine(y, self.slot, self.topk_w, self.T, self.H, self.k, self.out,
+    def combine(self, y: torch.Tensor, stream=None, out: Optional[torch.Tensor] = None):
+        out = self.out if out is None else out
+        B.ep_combine(y, self.slot, self.topk_w, self.T, self.H, self.k, out,
                      self.num_sms, self.copy_status, stream)
+        return out
 
-    def step(self, x, logits, bias, y, stream=None):
+    def step(self, x, logits, bias, y, stream=None, out=None):
         """route, layout, dispatch, then combine of the expert outputs y."""
         self.route(logits, bias, stream)
         self.layout(stream)
         self.dispatch(x, stream)
-        self.combine(y, stream)
-        return self.out
+        return self.combine(y, stream, out)
 
     def kernels_per_step(self) -> int:
         """Kernels one step launches: route, layout (count + slot, plus a
@@ -118,3 +119,54 @@ class EpPath:
         if st:
             raise B.EpError("ep path (device status %#x)" % st, B.EP_ERR_DEVICE)
         return st
+
+
+class EpHostPipeline:
+    """Runs batches that live in pinned host memory through an ``EpPath``
+    with the PCIe copies overlapped: while batch i computes, batch i+1's
+    inputs travel host -> device on one copy stream and batch i-1's result
+    travels device -> host on another.  Inputs and outputs are double
+    buffered on the device; the path's intermediate buffers are shared
+    because the compute stream runs one batch after the other.
+    """
+
+    def __init__(self, path: EpPath, device="cuda"):
+        dev = torch.device(device)
+        self.path = path
+        T, H, E = path.T, path.H, path.E
+        self.x = [torch.empty((T, H), device=dev, dtype=torch.bfloat16) for _ in range(2)]
+        self.logits = [torch.empty((T, E), device=dev, dtype=torch.float32) for _ in range(2)]
+        self.bias = [torch.empty(E, device=dev, dtype=torch.float32) for _ in range(2)]
+        self.out = [torch.empty((T, H), device=dev, dtype=torch.bfloat16) for _ in range(2)]
+        self.s_h2d = torch.cuda.Stream(dev)
+        self.s_comp = torch.cuda.Stream(dev)
+        self.s_d2h = torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.h2d_done, self.comp_done, self.d2h_done = ev(), ev(), ev()
+
+    def run(self, x_host, logits_host, bias_host, out_host, y):
+        """Enqueues every batch i: x_host[i], logits_host[i], bias_host[i]
+        (pinned CPU tensors) in, out_host[i] (pinned) out, with the expert
+        outputs ``y`` already on the device.  Returns without synchronising;
+        ``self.s_d2h`` carries the last copy."""
+        p = self.path
+        for i in range(len(x_host)):
+            b = i & 1
+            with torch.cuda.stream(self.s_h2d):
+                if i >= 2:  # buffer b was read by batch i-2's compute
+                    self.s_h2d.wait_event(self.comp_done[b])
+                self.x[b].copy_(x_host[i], non_blocking=True)
+                self.logits[b].copy_(logits_host[i], non_blocking=True)
+                self.bias[b].copy_(bias_host[i], non_blocking=True)
+                self.h2d_done[b].record(self.s_h2d)
+            self.s_comp.wait_event(self.h2d_done[b])
+            if i >= 2:      # out[b] was read by batch i-2's download
+                self.s_comp.wait_event(self.d2h_done[b])
+            with torch.cuda.stream(self.s_comp):
+                p.step(self.x[b], self.logits[b], self.bias[b], y, stream=self.s_comp,
+                       out=self.out[b])
+                self.comp_done[b].record(self.s_comp)
+            self.s_d2h.wait_event(self.comp_done[b])
+            with torch.cuda.stream(self.s_d2h):
+                out_host[i].copy_(self.out[b], non_blocking=True)
+                self.d2h_done[b].record(self.s_d2h)

@@ -468,3 +468,27 @@ def test_deterministic_across_runs_and_grids():
                                                 path.out)])
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+def test_host_pipeline_overlapped_batches():
+    """three different batches from pinned host memory through the
+    overlapped pipeline; every result equals the oracle's"""
+    from combine_ep_route_02_b200 import EpHostPipeline
+    cfg = CONFIGS["v3"].scaled(300)
+    wls = [Workload(cfg, seed=s) for s in (11, 12, 13)]
+    path = make_path(cfg, wls[0])
+    pipe = EpHostPipeline(path)
+    y = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=5)
+    xs = [w.x.pin_memory() for w in wls]
+    lgs = [w.logits.pin_memory() for w in wls]
+    bs = [w.bias.pin_memory() for w in wls]
+    outs = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in wls]
+    pipe.run(xs, lgs, bs, outs, y)
+    torch.cuda.synchronize()
+    yc = y.cpu()
+    for w, o in zip(wls, outs):
+        idx, wt, hard = oracle_route(cfg, w)
+        assert hard.sum() == 0
+        lay = oracle_layout(cfg, w, idx)
+        ref = oracle.combine(yc, lay["slot"], wt)
+        assert np.array_equal(u16(o), ref)
