@@ -203,6 +203,10 @@ def main():
     ap.add_argument("--config", default="v3", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    ap.add_argument("--schedule", default="micro", choices=["micro", "sequential"],
+                    help="micro: two micro-batches in flight (route+layout of batch i+1 "
+                         "overlap dispatch+combine of batch i); sequential: one step after "
+                         "the other on one stream")
     ap.add_argument("--num-sms", type=int, default=0)
     ap.add_argument("--ref-tokens", type=int, default=512,
                     help="tokens per oracle step (--impl reference and cpu_baseline)")
@@ -311,12 +315,39 @@ def main():
         s1[i].record(stream)
     torch.cuda.synchronize()
     barrier()
-    t_wall1 = time.perf_counter()
-    sampler.stop()
     path.check_status()
 
     step_ms = [a.elapsed_time(b) for a, b in zip(s0, s1)]
-    tot_ms = reduce_max(sum(step_ms), dist, "cuda")
+    seq_ms = reduce_max(sum(step_ms), dist, "cuda")
+    value_seq = tokens_per_s(cfg.T, world, K, seq_ms)
+
+    # the same K batches with two micro-batches in flight
+    micro_ms = None
+    if args.schedule == "micro":
+        from combine_ep_route_02_b200 import EpMicroBatchPipeline
+        from combine_ep_route_02_b200.path import EpPath as _EpPath
+
+        def make_path():
+            return _EpPath(cfg.T, cfg.H, cfg.E, cfg.n_group, cfg.topk_group, cfg.topk,
+                           cfg.routed_scale, cfg.renorm, cfg.R, cfg.fp8, phys_of=wl.phys_of,
+                           n_rep=wl.n_rep, num_sms=args.num_sms)
+        mb = EpMicroBatchPipeline(make_path)
+        mb.run([x] * args.warmup, [lg] * args.warmup, [bias] * args.warmup, [y] * args.warmup)
+        torch.cuda.synchronize()
+        barrier()
+        m0 = torch.cuda.Event(enable_timing=True)
+        m1 = torch.cuda.Event(enable_timing=True)
+        m0.record(mb.s_route)
+        mb.run([x] * K, [lg] * K, [bias] * K, [y] * K)
+        m1.record(mb.s_move)
+        torch.cuda.synchronize()
+        barrier()
+        mb.check_status()
+        micro_ms = reduce_max(m0.elapsed_time(m1), dist, "cuda")
+        del mb
+    t_wall1 = time.perf_counter()
+    sampler.stop()
+    tot_ms = micro_ms if micro_ms is not None else seq_ms
     value = tokens_per_s(cfg.T, world, K, tot_ms)
 
     peak, peak_kind = peak_hbm()
@@ -401,7 +432,12 @@ def main():
                        "l2": ("flushed before each step (256 MiB write, outside step events)"
                               if flush else
                               f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB moved per step)"),
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "schedule": ("two micro-batches in flight: route+layout of batch i+1 "
+                                    "on one stream overlap dispatch+combine of batch i on "
+                                    "another" if micro_ms is not None else
+                                    "sequential, one stream")},
+            "value_sequential": value_seq, "ms_per_step_sequential": seq_ms / K,
             "gpu_launches": path.kernels_per_step() * K,
             "roofline": roofline,
             "e2e": e2e,

@@ -25,4 +25,4 @@ from ._binding import (  # noqa: F401
     ep_workspace_size,
     lib,
 )
-from .path import EpHostPipeline, EpPath  # noqa: F401
+from .path import EpHostPipeline, EpMicroBatchPipeline, EpPath  # noqa: F401

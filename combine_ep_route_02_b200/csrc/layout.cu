@@ -186,24 +186,25 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
         // per expert: rows in tiles before this one, and in all tiles.  Four
         // consecutive lanes share a column, each summing every fourth tile
         // with four loads in flight, then combine by shuffles.
+        // NT <= 64, so a thread's share is at most 16 tiles: all its loads
+        // are issued before any is used (one L2 round trip)
         constexpr int PARTS = 4;
+        constexpr int PER = LAYOUT_FUSED_MAX_TILES / PARTS;
         for (int base = 0; base < a.P; base += LAYOUT_THREADS / PARTS) {
             const int p = base + (int)threadIdx.x / PARTS;
             const int part = threadIdx.x % PARTS;
             int before = 0, total = 0;
             if (p < a.P) {
-                for (int i0 = part; i0 < NT; i0 += 4 * PARTS) {
-                    int c[4];
+                int c[PER];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = i0 + u * PARTS;
-                        c[u] = (i < NT) ? __ldg(a.tile_cnt + (size_t)i * a.P + p) : 0;
-                    }
+                for (int u = 0; u < PER; ++u) {
+                    const int i = part + u * PARTS;
+                    c[u] = (i < NT) ? __ldg(a.tile_cnt + (size_t)i * a.P + p) : 0;
+                }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        before += (i0 + u * PARTS < tile) ? c[u] : 0;
-                        total += c[u];
-                    }
+                for (int u = 0; u < PER; ++u) {
+                    before += (part + u * PARTS < tile) ? c[u] : 0;
+                    total += c[u];
                 }
             }
 #pragma unroll
@@ -230,17 +231,13 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs 
     if (tile == 0) {
         if (FUSED) {
             for (int p = threadIdx.x; p < a.P; p += blockDim.x) a.cnt_expert[p] = eoff[p];
-            for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+            // one warp per rank, lanes over tiles (NT <= 64: two loads each)
+            for (int r = warp; r < a.R; r += LAYOUT_WARPS) {
                 int sum = 0;
-                for (int i0 = 0; i0 < NT; i0 += 8) {
-                    int c[8];
+                for (int i = lane; i < NT; i += 32) sum += __ldg(a.tile_tok + (size_t)i * a.R + r);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        c[u] = (i0 + u < NT) ? __ldg(a.tile_tok + (size_t)(i0 + u) * a.R + r) : 0;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) sum += c[u];
-                }
-                a.tok_rank[r] = sum;
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, off);
+                if (lane == 0) a.tok_rank[r] = sum;
             }
         }
         if (a.dev_status != nullptr && threadIdx.x < 32) {

@@ -170,3 +170,44 @@ class EpHostPipeline:
             with torch.cuda.stream(self.s_d2h):
                 out_host[i].copy_(self.out[b], non_blocking=True)
                 self.d2h_done[b].record(self.s_d2h)
+
+
+class EpMicroBatchPipeline:
+    """Two micro-batches in flight, as in the two-micro-batch overlap of
+    DeepSeek's and Perplexity's EP deployments: routing and layout of batch
+    i+1 (arithmetic- and latency-bound) run on one stream while dispatch and
+    combine of batch i (HBM-bound) run on another.  Each of the two
+    ``EpPath`` buffer sets serves every other batch; batch i+2 starts its
+    routing only after batch i has finished its combine.
+    """
+
+    def __init__(self, make_path, device="cuda"):
+        dev = torch.device(device)
+        self.paths = [make_path(), make_path()]
+        self.s_route = torch.cuda.Stream(dev)
+        self.s_move = torch.cuda.Stream(dev)
+        self.layout_done = [torch.cuda.Event() for _ in range(2)]
+        self.move_done = [torch.cuda.Event() for _ in range(2)]
+
+    def run(self, xs, logits, biases, ys):
+        """Enqueues batch i = (xs[i], logits[i], biases[i], expert outputs
+        ys[i]); results land in ``self.paths[i % 2].out``.  Returns without
+        synchronising; ``self.s_move`` carries the last combine."""
+        for i in range(len(xs)):
+            b = i & 1
+            p = self.paths[b]
+            if i >= 2:  # buffer set b is free once batch i-2 has combined
+                self.s_route.wait_event(self.move_done[b])
+            with torch.cuda.stream(self.s_route):
+                p.route(logits[i], biases[i], stream=self.s_route)
+                p.layout(stream=self.s_route)
+                self.layout_done[b].record(self.s_route)
+            self.s_move.wait_event(self.layout_done[b])
+            with torch.cuda.stream(self.s_move):
+                p.dispatch(xs[i], stream=self.s_move)
+                p.combine(ys[i], stream=self.s_move)
+                self.move_done[b].record(self.s_move)
+
+    def check_status(self):
+        for p in self.paths:
+            p.check_status()

@@ -492,3 +492,34 @@ def test_host_pipeline_overlapped_batches():
         lay = oracle_layout(cfg, w, idx)
         ref = oracle.combine(yc, lay["slot"], wt)
         assert np.array_equal(u16(o), ref)
+
+
+def test_micro_batch_pipeline():
+    """four different batches through the two-stream micro-batch schedule;
+    every batch's layout and result equal the oracle's"""
+    from combine_ep_route_02_b200 import EpMicroBatchPipeline
+    cfg = CONFIGS["skew"].scaled(700)
+    wls = [Workload(cfg, seed=s) for s in (21, 22, 23, 24)]
+    pipe = EpMicroBatchPipeline(lambda: make_path(cfg, wls[0]))
+    ys = [device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=30 + i) for i in range(4)]
+    outs = []
+    for i in range(4):  # one batch at a time so every result can be kept
+        pipe.run([wls[i].x.cuda()], [wls[i].logits.cuda()], [wls[i].bias.cuda()], [ys[i]])
+        torch.cuda.synchronize()
+        p = pipe.paths[0]
+        outs.append((u16(p.out), p.slot.cpu().numpy().copy()))
+    # every batch is laid out with the pipeline's replica map (batch 0's)
+    po, nr = wls[0].phys_of.numpy(), wls[0].n_rep.numpy()
+    for w, y, (o, sl) in zip(wls, ys, outs):
+        idx, wt, hard = oracle_route(cfg, w)
+        assert hard.sum() == 0
+        lay = oracle.layout(idx, cfg.E, cfg.n_phys, cfg.R, po, nr)
+        assert np.array_equal(sl, lay["slot"])
+        assert np.array_equal(o, oracle.combine(y.cpu(), lay["slot"], wt))
+    # all four enqueued at once: the overlapped schedule gives the same bytes
+    pipe.run([w.x.cuda() for w in wls], [w.logits.cuda() for w in wls],
+             [w.bias.cuda() for w in wls], ys)
+    torch.cuda.synchronize()
+    pipe.check_status()
+    assert np.array_equal(u16(pipe.paths[0].out), outs[2][0])
+    assert np.array_equal(u16(pipe.paths[1].out), outs[3][0])
