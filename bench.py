@@ -71,6 +71,39 @@ def tokens_per_s(T: int, world: int, steps: int, max_ms: float) -> float:
     return T * world * steps / (max_ms * 1e-3)
 
 
+def kernel_source_hash(*names) -> str:
+    """sha256 over the given kernel source files (package csrc/)."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "combine_ep_route_02_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(summary: str, workload: str, sources):
+    """DRAM bytes per launch recorded in profiles/<summary> for this
+    workload, or None when the kernel's sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            key, _, val = line[2:].partition(":")
+            fields[key.strip()] = val.strip().strip("`")
+    if fields.get("workload") != workload:
+        return None
+    if fields.get("source_sha256") != kernel_source_hash(*sources):
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -211,10 +244,15 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=512,
                     help="tokens per oracle step (--impl reference and cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens instead (small cases for "
+                         "profiler captures); 0 = the workload's own T")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     faulthandler.enable()
     cfg = CONFIGS[args.config]
+    if args.tokens > 0:
+        cfg = cfg.scaled(args.tokens)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
@@ -323,7 +361,9 @@ def main():
 
     # the same K batches with two micro-batches in flight
     micro_ms = None
-    if args.schedule == "micro":
+    # the two-stream schedule has no L2 flush between steps, so it is only
+    # timed when a step's data is larger than L2 anyway
+    if args.schedule == "micro" and not flush:
         from combine_ep_route_02_b200 import EpMicroBatchPipeline
         from combine_ep_route_02_b200.path import EpPath as _EpPath
 
@@ -362,7 +402,9 @@ def main():
                     "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy)"
                     if peak_kind == "measured" else "fallback 6650 GB/s",
-                    "traffic": None}
+                    "traffic": profiled_traffic(
+                        "combine_kernel_v3.md", f"{cfg.name} T={cfg.T}",
+                        ("combine.cu", "ep_device.cuh", "ep_internal.h"))}
         dc_ms = comb_ms + disp_ms
         route_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(s0, l0))
         layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(l0, d0))
