@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     ep_dispatch,
     ep_dispatch_layout,
     ep_route,
+    ep_route_layout,
     ep_workspace_size,
     lib,
 )

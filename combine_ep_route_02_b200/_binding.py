@@ -27,7 +27,7 @@ EP_DEV_TIMEOUT = 4
 
 # every symbol declared in include/ep.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
-           "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc")
+           "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout")
 
 
 class EpError(RuntimeError):
@@ -67,6 +67,9 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_layout_noalloc.argtypes = [P, I, I, I, I, I, P, P, I,
                                                  P, P, P, P, P, P, P, P, P, P]
         L.ep_dispatch_layout_noalloc.restype = I
+        L.ep_route_layout.argtypes = [P, P, I, RouteCfg, I, I, P, P, I,
+                                      P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.ep_route_layout.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -135,3 +138,14 @@ def ep_dispatch_layout_noalloc(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
         _ptr(topk_idx), T, k, E, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
         _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank), _ptr(rank_off), _ptr(tok_rank),
         _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(dev_status), _stream(stream)))
+
+
+def ep_route_layout(logits, bias, T, cfg: RouteCfg, P, R, phys_of, n_rep, max_rep, topk_idx,
+                    topk_w, cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
+                    src, workspace, dev_status, stream=None):
+    """ep_route followed by ep_dispatch_layout (one kernel for small batches)."""
+    _check("ep_route_layout", lib().ep_route_layout(
+        _ptr(logits), _ptr(bias), T, cfg, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
+        _ptr(topk_idx), _ptr(topk_w), _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank),
+        _ptr(rank_off), _ptr(tok_rank), _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace),
+        _ptr(dev_status), _stream(stream)))

@@ -85,8 +85,13 @@ size_t ep_workspace_size(int T, int k, int P, int R)
     return layout_workspace_bytes(T, k, P, R);
 }
 
-ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
-                   int32_t *topk_idx, float *topk_w, ep_stream_t stream)
+}  // extern "C"
+
+namespace ep {
+namespace {
+
+ep_status check_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                      int32_t *topk_idx, float *topk_w)
 {
     const int E = cfg.num_experts, G = cfg.n_group, Kg = cfg.topk_group, k = cfg.topk;
     if (T < 0 || E < 1 || G < 1 || Kg < 1 || k < 1) return EP_ERR_INVALID;
@@ -97,16 +102,14 @@ ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg c
     if (T > 0 && (!logits || !topk_idx || !topk_w)) return EP_ERR_INVALID;
     if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
         return EP_ERR_INVALID;
-    RouteArgs a{logits, bias, T, E, G, Kg, k, cfg.routed_scale, cfg.renorm != 0, topk_idx, topk_w};
-    return from_cuda(launch_route(a, reinterpret_cast<cudaStream_t>(stream)));
+    return EP_OK;
 }
 
-ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
-                             const int32_t *phys_of, const int32_t *n_rep, int max_rep,
-                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
-                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
-                             int32_t *slot, int32_t *src, void *workspace,
-                             int32_t *dev_status, ep_stream_t stream)
+ep_status check_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                       int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank, int32_t *slot,
+                       int32_t *src, void *workspace, int32_t *dev_status)
 {
     if (T < 0 || k < 1 || E < 1 || P < 1 || R < 1) return EP_ERR_INVALID;
     if (P % R != 0) return EP_ERR_INVALID;
@@ -120,15 +123,85 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
     if (!aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(slot, 4) || !aligned(src, 4) ||
         !aligned(dev_status, 4))
         return EP_ERR_INVALID;
+    return EP_OK;
+}
+
+LayoutArgs layout_args(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                       int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank, int32_t *slot,
+                       int32_t *src, void *workspace, int32_t *dev_status)
+{
     const int NT = layout_tiles(T, k, P);
     char *ws = static_cast<char *>(workspace);
     const size_t o1 = align256((size_t)NT * P * sizeof(int32_t));
     const size_t o2 = o1 + align256((size_t)NT * R * sizeof(int32_t));
-    LayoutArgs a{topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
-                 cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
-                 reinterpret_cast<int32_t *>(ws), reinterpret_cast<int32_t *>(ws + o1),
-                 reinterpret_cast<int32_t *>(ws + o2), dev_status, layout_tile_tokens(T, k, P), NT, layout_hist_warps(P)};
+    return LayoutArgs{topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
+                      cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
+                      reinterpret_cast<int32_t *>(ws), reinterpret_cast<int32_t *>(ws + o1),
+                      reinterpret_cast<int32_t *>(ws + o2), dev_status,
+                      layout_tile_tokens(T, k, P), NT, layout_hist_warps(P)};
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" {
+
+ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                   int32_t *topk_idx, float *topk_w, ep_stream_t stream)
+{
+    const ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
+    if (st != EP_OK) return st;
+    RouteArgs a{logits, bias, T, cfg.num_experts, cfg.n_group, cfg.topk_group, cfg.topk,
+                cfg.routed_scale, cfg.renorm != 0, topk_idx, topk_w};
+    return from_cuda(launch_route(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                             const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
+                             int32_t *slot, int32_t *src, void *workspace,
+                             int32_t *dev_status, ep_stream_t stream)
+{
+    const ep_status st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
+                                      cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
+                                      in_rank, slot, src, workspace, dev_status);
+    if (st != EP_OK) return st;
+    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
+                                     expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
+                                     src, workspace, dev_status);
     return from_cuda(launch_layout(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                          int P, int R, const int32_t *phys_of, const int32_t *n_rep,
+                          int max_rep, int32_t *topk_idx, float *topk_w, int32_t *cnt_expert,
+                          int32_t *expert_off, int32_t *rows_rank, int32_t *rank_off,
+                          int32_t *tok_rank, uint8_t *in_rank, int32_t *slot, int32_t *src,
+                          void *workspace, int32_t *dev_status, ep_stream_t stream)
+{
+    ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
+    if (st != EP_OK) return st;
+    const int E = cfg.num_experts, k = cfg.topk;
+    st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert, expert_off,
+                      rows_rank, rank_off, tok_rank, in_rank, slot, src, workspace, dev_status);
+    if (st != EP_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const RouteArgs r{logits, bias, T, E, cfg.n_group, cfg.topk_group, k, cfg.routed_scale,
+                      cfg.renorm != 0, topk_idx, topk_w};
+    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
+                                     expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
+                                     src, workspace, dev_status);
+    if (small_route_layout_ok(T, k, P)) {
+        int *done = reinterpret_cast<int *>(static_cast<char *>(workspace) +
+                                            layout_workspace_core(T, k, P, R));
+        return from_cuda(launch_route_layout_small(r, a, done, s));
+    }
+    const cudaError_t e = launch_route(r, s);
+    if (e != cudaSuccess) return EP_ERR_CUDA;
+    return from_cuda(launch_layout(a, s));
 }
 
 ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,

@@ -100,13 +100,22 @@ inline int layout_tiles(int T, int k, int P)
     return (T + tt - 1) / tt;
 }
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
-// workspace bytes: tile_cnt, tile_tok, tile_bad, each 256-byte aligned
-inline size_t layout_workspace_bytes(int T, int k, int P, int R)
+// workspace bytes: tile_cnt, tile_tok, tile_bad, each 256-byte aligned, then
+// 256 bytes holding the fused small-batch kernel's completion counter
+inline size_t layout_workspace_core(int T, int k, int P, int R)
 {
     const size_t NT = (size_t)layout_tiles(T > 0 ? T : 1, k, P);
     return align256(NT * P * sizeof(int32_t)) + align256(NT * R * sizeof(int32_t)) +
            align256(NT * sizeof(int32_t));
 }
+inline size_t layout_workspace_bytes(int T, int k, int P, int R)
+{
+    return layout_workspace_core(T, k, P, R) + 256;
+}
+
+// Fused routing + layout for small batches (one kernel; see fused.cu).
+constexpr int SMALL_MAX_PAIRS = 4096;
+constexpr int SMALL_MAX_PHYS = 1024;
 
 // Programmatic dependent launch: every kernel of the path is launched with
 // programmatic stream serialisation, calls pdl_launch_dependents() so the
@@ -131,6 +140,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t s);
+bool small_route_layout_ok(int T, int k, int P);
+cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *done,
+                                      cudaStream_t s);
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);

@@ -1,0 +1,313 @@
+// Sigmoid-gated, group-limited top-k routing, device side: one warp per token.
+// Included by the routing kernel and by the fused small-batch kernel.
+//
+// DeepSeek group-limited routing (DeepSeek Open Infra day-4 summary, EPLB
+// section) with plain top-k as its one-group special case (Perplexity blog,
+// section "MoE Router").  Lane l holds experts [l*EPL, (l+1)*EPL).
+//
+// Every arg-max (groups, then each of the k experts) is two warp reductions
+// on integers: redux.sync max over an order-preserving 32-bit image of the
+// fp32 key, then redux.sync min over the indices of the lanes holding that
+// maximum, which is exactly the (key desc, index asc) order.  Keys are never
+// -0.0 or NaN here (s >= 0, and s + b rounds an exact zero to +0), so the
+// integer order equals the fp32 order.
+//
+// When a group is a power-of-two number of whole lanes (E/G a multiple of
+// EPL), each lane sits in one group and the group top-2 is a butterfly over
+// that group's lanes only; otherwise a general loop over groups is used.
+//
+// The fp64 sigmoid uses a table-driven exp and a Newton reciprocal rather
+// than the library exp and IEEE division: its fp64 value is within a few
+// ulps of the exact one, far inside the 2^-47 relative distance from an fp32
+// rounding midpoint below which another fp64 evaluation may round the other
+// way, so the fp32 result is the same as any such evaluation's.
+#pragma once
+
+#include <math.h>
+
+#include "ep_device.cuh"
+#include "ep_internal.h"
+
+namespace ep {
+namespace route_impl {
+
+// fp32 -> uint32 with the same order (for finite, non-NaN values; -0 and +0
+// map to different images, which never matters for the keys used here).
+EP_DEV uint32_t ordered(float f)
+{
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+constexpr uint32_t NONE = 0u;  // below the image of every float, -inf included
+
+// 2^(j/64) for j = 0..63, each correctly rounded to double
+__constant__ double kExp2Frac[64] = {
+    0x1.0000000000000p+0, 0x1.02c9a3e778061p+0, 0x1.059b0d3158574p+0, 0x1.0874518759bc8p+0,
+    0x1.0b5586cf9890fp+0, 0x1.0e3ec32d3d1a2p+0, 0x1.11301d0125b51p+0, 0x1.1429aaea92de0p+0,
+    0x1.172b83c7d517bp+0, 0x1.1a35beb6fcb75p+0, 0x1.1d4873168b9aap+0, 0x1.2063b88628cd6p+0,
+    0x1.2387a6e756238p+0, 0x1.26b4565e27cddp+0, 0x1.29e9df51fdee1p+0, 0x1.2d285a6e4030bp+0,
+    0x1.306fe0a31b715p+0, 0x1.33c08b26416ffp+0, 0x1.371a7373aa9cbp+0, 0x1.3a7db34e59ff7p+0,
+    0x1.3dea64c123422p+0, 0x1.4160a21f72e2ap+0, 0x1.44e086061892dp+0, 0x1.486a2b5c13cd0p+0,
+    0x1.4bfdad5362a27p+0, 0x1.4f9b2769d2ca7p+0, 0x1.5342b569d4f82p+0, 0x1.56f4736b527dap+0,
+    0x1.5ab07dd485429p+0, 0x1.5e76f15ad2148p+0, 0x1.6247eb03a5585p+0, 0x1.6623882552225p+0,
+    0x1.6a09e667f3bcdp+0, 0x1.6dfb23c651a2fp+0, 0x1.71f75e8ec5f74p+0, 0x1.75feb564267c9p+0,
+    0x1.7a11473eb0187p+0, 0x1.7e2f336cf4e62p+0, 0x1.82589994cce13p+0, 0x1.868d99b4492edp+0,
+    0x1.8ace5422aa0dbp+0, 0x1.8f1ae99157736p+0, 0x1.93737b0cdc5e5p+0, 0x1.97d829fde4e50p+0,
+    0x1.9c49182a3f090p+0, 0x1.a0c667b5de565p+0, 0x1.a5503b23e255dp+0, 0x1.a9e6b5579fdbfp+0,
+    0x1.ae89f995ad3adp+0, 0x1.b33a2b84f15fbp+0, 0x1.b7f76f2fb5e47p+0, 0x1.bcc1e904bc1d2p+0,
+    0x1.c199bdd85529cp+0, 0x1.c67f12e57d14bp+0, 0x1.cb720dcef9069p+0, 0x1.d072d4a07897cp+0,
+    0x1.d5818dcfba487p+0, 0x1.da9e603db3285p+0, 0x1.dfc97337b9b5fp+0, 0x1.e502ee78b3ff6p+0,
+    0x1.ea4afa2a490dap+0, 0x1.efa1bee615a27p+0, 0x1.f50765b6e4540p+0, 0x1.fa7c1819e90d8p+0,
+};
+
+// exp(y) for -700 <= y <= 700 in fp64, table-driven after P. T. P. Tang,
+// "Table-driven implementation of the exponential function in IEEE
+// floating-point arithmetic", ACM TOMS 15(2), 1989: y = (64 m + j) ln2/64 + r
+// with |r| <= ln2/128, exp(y) = 2^m * 2^(j/64) * (1 + p(r)), p the degree-6
+// Taylor polynomial of e^r - 1 (truncation below 2^-64).  ln2/64 is split so
+// that N * L1 is exact for |N| < 2^17.  Error: a few units in the last place.
+EP_DEV double exp_table(double y, const double *tab)
+{
+    const double K = 0x1.71547652b82fep+6;   // 64 / ln 2
+    const double L1 = 0x1.62e42fefa0000p-7;  // high 36 bits of ln2 / 64
+    const double L2 = 0x1.cf79abc9e3b3ap-46; // ln2 / 64 - L1
+    const double Nd = rint(y * K);
+    const int N = (int)Nd;
+    double r = fma(-Nd, L1, y);
+    r = fma(-Nd, L2, r);
+    double p = fma(r, 1.0 / 720.0, 1.0 / 120.0);
+    p = fma(r, p, 1.0 / 24.0);
+    p = fma(r, p, 1.0 / 6.0);
+    p = fma(r, p, 0.5);
+    p = fma(r, p, 1.0);
+    p = p * r;
+    const double t = tab[N & 63];
+    const double e = fma(t, p, t);
+    return e * __hiloint2double((1023 + (N >> 6)) << 20, 0);
+}
+
+// s = fp32(1 / (1 + exp(-x))) from an fp64 evaluation accurate to a few
+// fp64 ulps (the reciprocal: a hardware estimate and two Newton steps).
+EP_DEV float sigmoid_f32(float x, const double *tab)
+{
+    double y = -(double)x;
+    if (y > 700.0) return 0.0f;    // s < e^-700 rounds to +0 in fp32
+    if (y < -700.0) y = -700.0;    // 1 + e^y rounds to 1 either way
+    const double d = 1.0 + exp_table(y, tab);
+    double z;
+    asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(z) : "d"(d));
+    z = fma(z, fma(-d, z, 1.0), z);
+    z = fma(z, fma(-d, z, 1.0), z);
+    return __double2float_rn(z);
+}
+
+// winner of (key desc, index asc) over the warp; every lane gets it
+EP_DEV int warp_pick(uint32_t key, int idx)
+{
+    const uint32_t kmax = __reduce_max_sync(FULL_MASK, key);
+    const uint32_t cand = (key == kmax) ? (uint32_t)idx : 0xffffffffu;
+    return (int)__reduce_min_sync(FULL_MASK, cand);
+}
+
+// Routes tokens t_first, t_first + t_stride, ... < T with the calling warp.
+// tab: the 2^(j/64) table in shared memory.
+template <int EPL>
+EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restrict__ bias, int T,
+                         int E, int G, int Kg, int k, float scale, int renorm, int vec4,
+                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                         const double *tab, int t_first, int t_stride)
+{
+    const int lane = threadIdx.x & 31;
+    const int e0 = lane * EPL;
+    const int gs = E / G;
+    // each lane lies inside one group when gs is a multiple of EPL; the
+    // butterfly below also needs the group's lane count to be a power of two
+    const int lpg = gs / EPL;
+    const bool aligned = (gs % EPL) == 0 && (lpg & (lpg - 1)) == 0;
+    const int lanes_per_group = aligned ? lpg : 0;
+    const int my_group = (e0 < E) ? e0 / gs : -1;        // valid when aligned
+
+    float b[EPL];
+    int gid[EPL];  // token-invariant group of each held expert (-1: none)
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const bool v = e0 + i < E;
+        b[i] = (bias != nullptr && v) ? bias[e0 + i] : 0.0f;
+        gid[i] = v ? (e0 + i) / gs : -1;
+    }
+
+    for (int t = t_first; t < T; t += t_stride) {
+        const float *row = logits + (size_t)t * E;
+        float x[EPL];
+        if (EPL % 4 == 0 && vec4) {
+#pragma unroll
+            for (int q = 0; q < EPL / 4; ++q) {
+                // E % 4 == 0, so a quad is either wholly inside the row or not
+                float4 v = (e0 + 4 * q < E)
+                               ? __ldg(reinterpret_cast<const float4 *>(row + e0) + q)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[4 * q + 0] = v.x;
+                x[4 * q + 1] = v.y;
+                x[4 * q + 2] = v.z;
+                x[4 * q + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) x[i] = (e0 + i < E) ? __ldg(row + e0 + i) : 0.0f;
+        }
+
+        // s = fp32(1 / (1 + exp(-x))) evaluated in fp64; key = fp32(s + b)
+        float s[EPL];
+        uint32_t key[EPL];
+        uint32_t live = 0;  // bit i: expert e0+i exists and is still eligible
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            if (e0 + i < E) {
+                s[i] = sigmoid_f32(x[i], tab);
+                key[i] = ordered(__fadd_rn(__fadd_rn(s[i], b[i]), 0.0f));
+                live |= 1u << i;
+            } else {
+                s[i] = 0.0f;
+                key[i] = NONE;
+            }
+        }
+
+        if (G > 1) {
+            // group score = fp32 sum of the two largest keys in the group
+            uint32_t chosen = 0;
+            if (aligned) {
+                float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) {
+                    if (!((live >> i) & 1u)) continue;
+                    const float v = __fadd_rn(s[i], b[i]);
+                    if (v > a1) {
+                        a2 = a1;
+                        a1 = v;
+                    } else if (v > a2) {
+                        a2 = v;
+                    }
+                }
+                // butterfly over the lanes of this group (they are contiguous
+                // and start at a multiple of lanes_per_group)
+                for (int off = 1; off < lanes_per_group; off <<= 1) {
+                    const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                    const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                    const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                    a1 = fmaxf(a1, o1);
+                    a2 = n2;
+                }
+                const uint32_t my_score =
+                    (my_group >= 0) ? ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f)) : NONE;
+                for (int r = 0; r < Kg; ++r) {
+                    const bool cand = my_group >= 0 && !((chosen >> my_group) & 1u);
+                    const int g = warp_pick(cand ? my_score : NONE, cand ? my_group : 0x7fffffff);
+                    chosen |= 1u << g;
+                }
+            } else {
+                uint32_t my_score = NONE;  // lane g keeps the score of group g
+                for (int g = 0; g < G; ++g) {
+                    float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) {
+                        if (gid[i] != g) continue;
+                        const float v = __fadd_rn(s[i], b[i]);
+                        if (v > a1) {
+                            a2 = a1;
+                            a1 = v;
+                        } else if (v > a2) {
+                            a2 = v;
+                        }
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {
+                        const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                        const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                        const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                        a1 = fmaxf(a1, o1);
+                        a2 = n2;
+                    }
+                    if (lane == g) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
+                }
+                for (int r = 0; r < Kg; ++r) {
+                    const bool cand = lane < G && !((chosen >> lane) & 1u);
+                    const int g = warp_pick(cand ? my_score : NONE, cand ? lane : 0x7fffffff);
+                    chosen |= 1u << g;
+                }
+            }
+            if (aligned) {
+                // the lane's experts share one group
+                if (my_group >= 0 && !((chosen >> my_group) & 1u))
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) key[i] = NONE;
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) key[i] = NONE;
+            }
+        }
+
+        // lane-local best: the first (lowest index) of the largest keys;
+        // excluded and taken experts hold NONE, below every real key
+        uint32_t best_k = NONE;
+        int best_i = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (key[i] > best_k) {
+                best_k = key[i];
+                best_i = e0 + i;
+            }
+
+        int sel_idx = 0;
+        float sel_s = 0.0f;
+        for (int r = 0; r < k; ++r) {
+            const int e = warp_pick(best_k, best_i);
+            const int owner = e / EPL;  // k <= eligible experts, so e is real
+            float sv = 0.0f;
+            if (lane == owner) {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (e0 + i == e) {
+                        sv = s[i];
+                        key[i] = NONE;
+                    }
+                best_k = NONE;
+                best_i = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (key[i] > best_k) {
+                        best_k = key[i];
+                        best_i = e0 + i;
+                    }
+            }
+            sv = __shfl_sync(FULL_MASK, sv, owner);
+            if (lane == r) {
+                sel_idx = e;
+                sel_s = sv;
+            }
+        }
+
+        float w = sel_s;
+        if (renorm) {
+            float sum = 0.0f;
+            for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(FULL_MASK, sel_s, j));
+            if (sum != 0.0f) w = __fdiv_rn(w, sum);
+        }
+        w = __fmul_rn(w, scale);
+        if (lane < k) {
+            topk_idx[(size_t)t * k + lane] = sel_idx;
+            topk_w[(size_t)t * k + lane] = w;
+        }
+    }
+}
+
+
+// copies the exp table into shared memory (all threads of the block call it)
+EP_DEV void load_exp_table(double *tab)
+{
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) tab[i] = kExp2Frac[i];
+}
+
+}  // namespace route_impl
+}  // namespace ep

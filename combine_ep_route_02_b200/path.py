@@ -79,6 +79,14 @@ class EpPath:
                              self.in_rank, self.slot, self.src, self.workspace,
                              self.dev_status, stream)
 
+    def route_layout(self, logits: torch.Tensor, bias: Optional[torch.Tensor], stream=None):
+        """route then layout in one call (one kernel for small batches)"""
+        B.ep_route_layout(logits, bias, self.T, self.cfg, self.P, self.R, self.phys_of,
+                          self.n_rep, self.max_rep, self.topk_idx, self.topk_w,
+                          self.cnt_expert, self.expert_off, self.rows_rank, self.rank_off,
+                          self.tok_rank, self.in_rank, self.slot, self.src, self.workspace,
+                          self.dev_status, stream)
+
     def dispatch(self, x: torch.Tensor, stream=None):
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
                       self.recv_scale, self.num_sms, self.copy_status, stream)
@@ -91,8 +99,7 @@ class EpPath:
 
     def step(self, x, logits, bias, y, stream=None, out=None):
         """route, layout, dispatch, then combine of the expert outputs y."""
-        self.route(logits, bias, stream)
-        self.layout(stream)
+        self.route_layout(logits, bias, stream)
         self.dispatch(x, stream)
         return self.combine(y, stream, out)
 
@@ -103,6 +110,8 @@ class EpPath:
         tiles can grow, capped by the slot kernel's shared memory)."""
         if self.T == 0:
             return 1
+        if self.T * self.k <= 4096 and self.P <= 1024:
+            return 3  # fused route + layout, dispatch, combine
         tt = max(64, min(512, -(-self.T // 64)))
         hw = 32
         while hw > 1 and hw * self.P > 32768:
@@ -199,8 +208,7 @@ class EpMicroBatchPipeline:
             if i >= 2:  # buffer set b is free once batch i-2 has combined
                 self.s_route.wait_event(self.move_done[b])
             with torch.cuda.stream(self.s_route):
-                p.route(logits[i], biases[i], stream=self.s_route)
-                p.layout(stream=self.s_route)
+                p.route_layout(logits[i], biases[i], stream=self.s_route)
                 self.layout_done[b].record(self.s_route)
             self.s_move.wait_event(self.layout_done[b])
             with torch.cuda.stream(self.s_move):

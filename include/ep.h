@@ -155,6 +155,25 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
                              int32_t *dev_status, ep_stream_t stream);
 
 /*
+ * Routing followed by the dispatch layout, in one call (the cached-handle /
+ * low-latency decode use of the DeepEP V2 summary, section "Usage for
+ * training, prefill and decoding").  Arguments are those of ep_route and
+ * ep_dispatch_layout (E = cfg.num_experts, k = cfg.topk); the results are
+ * identical to calling the two in sequence.  For small batches
+ * (T * k <= 4096 and P <= 1024) a single kernel does both: its routing blocks
+ * count themselves done on a counter in the workspace, and the last one lays
+ * out the whole batch, so no block waits for another.  Larger batches run the
+ * two calls' kernels back to back.  workspace: ep_workspace_size(T, k, P, R)
+ * bytes, 256-byte aligned.
+ */
+ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                          int P, int R, const int32_t *phys_of, const int32_t *n_rep,
+                          int max_rep, int32_t *topk_idx, float *topk_w, int32_t *cnt_expert,
+                          int32_t *expert_off, int32_t *rows_rank, int32_t *rank_off,
+                          int32_t *tok_rank, uint8_t *in_rank, int32_t *slot, int32_t *src,
+                          void *workspace, int32_t *dev_status, ep_stream_t stream);
+
+/*
  * Dispatch (permute, optionally with fused 1x128 FP8 quantisation).
  *
  *   x_bf16      bf16 [T, H], 16-byte aligned; H % 8 == 0 (H % 128 == 0 for fp8)

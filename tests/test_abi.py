@@ -44,9 +44,10 @@ def test_status_strings(lib):
 def test_workspace_size(lib):
     # NT tiles of max(64, ceil(T/64)) tokens; [NT][P] + [NT][R] + [NT] int32,
     # each rounded up to 256 bytes
-    assert ep.ep_workspace_size(8192, 8, 256, 8) == 64 * 256 * 4 + 2048 + 256
-    assert ep.ep_workspace_size(1, 8, 288, 32) == 1280 + 256 + 256
-    assert ep.ep_workspace_size(16384, 8, 288, 32) == 64 * 288 * 4 + 64 * 32 * 4 + 256
+    # (+ 256 bytes for the fused small-batch kernel's completion counter)
+    assert ep.ep_workspace_size(8192, 8, 256, 8) == 64 * 256 * 4 + 2048 + 256 + 256
+    assert ep.ep_workspace_size(1, 8, 288, 32) == 1280 + 256 + 256 + 256
+    assert ep.ep_workspace_size(16384, 8, 288, 32) == 64 * 288 * 4 + 64 * 32 * 4 + 256 + 256
     assert ep.ep_workspace_size(0, 8, 256, 8) > 0
     assert ep.ep_workspace_size(-1, 8, 256, 8) == 0
     assert ep.ep_workspace_size(10, 0, 256, 8) == 0

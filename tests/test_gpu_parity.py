@@ -523,3 +523,32 @@ def test_micro_batch_pipeline():
     pipe.check_status()
     assert np.array_equal(u16(pipe.paths[0].out), outs[2][0])
     assert np.array_equal(u16(pipe.paths[1].out), outs[3][0])
+
+
+@pytest.mark.parametrize("name,T", [("v3_decode", 256), ("v3_decode", 1), ("v3_decode", 77),
+                                    ("tiny", 128), ("skew", 512), ("ds16b", 682),
+                                    ("v3", 513), ("skew", 3000)])
+def test_route_layout_fused_equals_two_calls(name, T):
+    """ep_route_layout (one kernel while T*k <= 4096) gives the bytes of
+    ep_route + ep_dispatch_layout and of the oracle"""
+    cfg = CONFIGS[name].scaled(T)
+    wl = Workload(cfg, seed=40 + T)
+    a, b = make_path(cfg, wl), make_path(cfg, wl)
+    lg, bs = wl.logits.cuda(), wl.bias.cuda()
+    a.route(lg, bs)
+    a.layout()
+    b.dev_status.fill_(-1)
+    b.route_layout(lg, bs)
+    torch.cuda.synchronize()
+    for n in ("topk_idx", "topk_w", "cnt_expert", "expert_off", "rows_rank", "rank_off",
+              "tok_rank", "in_rank", "slot", "src", "dev_status"):
+        assert torch.equal(getattr(a, n), getattr(b, n)), n
+    idx, w, hard = oracle_route(cfg, wl)
+    assert hard.sum() == 0
+    assert np.array_equal(b.topk_idx.cpu().numpy(), idx)
+    lay = oracle_layout(cfg, wl, idx)
+    assert np.array_equal(b.slot.cpu().numpy(), lay["slot"])
+    # a second call on the same workspace (the completion counter is reset)
+    b.route_layout(lg, bs)
+    torch.cuda.synchronize()
+    assert torch.equal(a.slot, b.slot)
