@@ -2,7 +2,7 @@
 """Throughput of the MoE routing -> layout -> FP8 dispatch -> combine path.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3]
-                    [--impl ours|reference] [--graph]
+                    [--impl ours|reference] [--schedule micro|sequential]
 
 One step = route + dispatch layout + dispatch + combine over one batch of the
 named workload (default: DeepSeek-V3 prefill shape, T=8192 tokens, H=7168,
@@ -235,7 +235,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
     ap.add_argument("--schedule", default="micro", choices=["micro", "sequential"],
                     help="micro: two micro-batches in flight (route+layout of batch i+1 "
                          "overlap dispatch+combine of batch i); sequential: one step after "
@@ -286,7 +285,15 @@ def main():
     ab = algorithmic_bytes(cfg)
     step_bytes = sum(ab.values())
     flush = step_bytes < 2 * L2_BYTES
-    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda") if flush else None
+    # L2 flush between steps: write 256 MiB, then read another 256 MiB, so
+    # that L2 holds none of the step's data and no dirty lines whose write-back
+    # the next step would pay for
+    flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda") if flush else None
+    flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda") if flush else None
+
+    def flush_l2(i):
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
 
     def barrier():
         if dist is not None:
@@ -295,71 +302,74 @@ def main():
     def step():
         path.step(x, lg, bias, y)
 
-    graph = None
-    if args.graph:
-        s = torch.cuda.Stream()
-        s.wait_stream(stream)
-        with torch.cuda.stream(s):
-            step()
-        stream.wait_stream(s)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step()
-
-    def run_step():
-        if graph is not None:
-            graph.replay()
-        else:
-            step()
-
     for _ in range(args.warmup):
-        run_step()
+        step()
     torch.cuda.synchronize()
     path.check_status()
 
-    # kernel-level events (combine = dominant kernel) are recorded inside the
-    # timed region on the launching stream; they need eager launches
-    kev = graph is None
     K = args.steps
-    c0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
-    c1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
-    l0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
-    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
-    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if kev else []
-    s0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    s1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
 
+    def events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def total_ms(a, b):
+        return reduce_max(sum(x.elapsed_time(y) for x, y in zip(a, b)), dist, "cuda")
+
+    s0, s1, d0, d1, c0, c1 = events(), events(), events(), events(), events(), events()
     sampler = ClockSampler(local)
     sampler.start()
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
+
+    # 1. eager launches on one stream, events around route+layout, dispatch
+    #    and combine (the per-kernel attribution and the roofline)
     for i in range(K):
         if flush:
-            flush_buf.fill_(i & 0xFF)  # evict the previous step's data from L2
+            flush_l2(i)  # evict the previous step's data from L2
         s0[i].record(stream)
-        if kev:
-            path.route(lg, bias)
-            l0[i].record(stream)
-            path.layout()
-            d0[i].record(stream)
-            path.dispatch(x)
-            d1[i].record(stream)
-            c0[i].record(stream)
-            path.combine(y)
-            c1[i].record(stream)
-        else:
-            run_step()
+        path.route_layout(lg, bias)
+        d0[i].record(stream)
+        path.dispatch(x)
+        d1[i].record(stream)
+        c0[i].record(stream)
+        path.combine(y)
+        c1[i].record(stream)
         s1[i].record(stream)
     torch.cuda.synchronize()
     barrier()
     path.check_status()
+    eager_ms = total_ms(s0, s1)
 
-    step_ms = [a.elapsed_time(b) for a, b in zip(s0, s1)]
-    seq_ms = reduce_max(sum(step_ms), dist, "cuda")
+    # 2. the same step captured once as a CUDA graph and replayed: no host
+    #    launch cost per kernel (what bounds small batches when eager)
+    gs = torch.cuda.Stream()
+    gs.wait_stream(stream)
+    with torch.cuda.stream(gs):
+        step()
+    stream.wait_stream(gs)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    g0, g1 = events(), events()
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(K):
+        if flush:
+            flush_l2(i)
+        g0[i].record(stream)
+        graph.replay()
+        g1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    path.check_status()
+    graph_ms = total_ms(g0, g1)
+    seq_ms = graph_ms
     value_seq = tokens_per_s(cfg.T, world, K, seq_ms)
 
-    # the same K batches with two micro-batches in flight
+    # 3. the same K batches with two micro-batches in flight
     micro_ms = None
     # the two-stream schedule has no L2 flush between steps, so it is only
     # timed when a step's data is larger than L2 anyway
@@ -393,7 +403,7 @@ def main():
     peak, peak_kind = peak_hbm()
     roofline = None
     extra = {}
-    if kev:
+    if True:
         comb_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(c0, c1))
         disp_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(d0, d1))
         comb_gbs = ab["combine"] / (comb_ms * 1e-3) / 1e9
@@ -406,10 +416,9 @@ def main():
                         "combine_kernel_v3.md", f"{cfg.name} T={cfg.T}",
                         ("combine.cu", "ep_device.cuh", "ep_internal.h"))}
         dc_ms = comb_ms + disp_ms
-        route_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(s0, l0))
-        layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(l0, d0))
+        rl_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(s0, d0))
         extra = {
-            "route_us": route_ms * 1e3, "layout_us": layout_ms * 1e3,
+            "route_layout_us": rl_ms * 1e3,
             "dispatch_us": disp_ms * 1e3, "combine_us": comb_ms * 1e3,
             "dispatch_gbs": disp_gbs, "combine_gbs": comb_gbs,
             "dispatch_combine_tokens_per_s": cfg.T * world / (dc_ms * 1e-3),
@@ -470,7 +479,7 @@ def main():
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
                        "P": cfg.n_phys, "R": cfg.R, "n_group": cfg.n_group,
                        "topk_group": cfg.topk_group, "topk": cfg.topk, "fp8": cfg.fp8,
-                       "routed_scale": cfg.routed_scale, "cuda_graph": graph is not None,
+                       "routed_scale": cfg.routed_scale, "cuda_graph": micro_ms is None,
                        "l2": ("flushed before each step (256 MiB write, outside step events)"
                               if flush else
                               f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB moved per step)"),
@@ -478,9 +487,13 @@ def main():
                        "schedule": ("two micro-batches in flight: route+layout of batch i+1 "
                                     "on one stream overlap dispatch+combine of batch i on "
                                     "another" if micro_ms is not None else
-                                    "sequential, one stream")},
+                                    "sequential, one stream, step replayed as a CUDA graph")},
             "value_sequential": value_seq, "ms_per_step_sequential": seq_ms / K,
+            "value_sequential_eager": tokens_per_s(cfg.T, world, K, eager_ms),
+            "ms_per_step_sequential_eager": eager_ms / K,
             "gpu_launches": path.kernels_per_step() * K,
+            "gpu_launches_note": "per timed pass of K steps (each of the eager, graph and "
+                                 "micro-batch passes launches this many)",
             "roofline": roofline,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -489,8 +502,7 @@ def main():
             **extra,
         }
         print(json.dumps(line), flush=True)
-    if graph is not None:
-        del graph
+    del graph
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

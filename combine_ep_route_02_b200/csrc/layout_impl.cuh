@@ -61,15 +61,34 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
     __syncthreads();
 
     const int epr = a.P / a.R;
-    for (int i = threadIdx.x; i < nt * a.R; i += blockDim.x) {
-        const int tl = i / a.R, r = i - tl * a.R;
-        int hit = 0;
-        for (int j = 0; j < a.k; ++j) {
-            const int p = pp[tl * a.k + j];
-            hit |= (p >= 0 && p / epr == r);
+    if (a.R <= 64) {
+        // thread per token: the set of ranks it reaches as a bit mask, then
+        // its in_rank row byte by byte (consecutive threads write
+        // neighbouring rows)
+        for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
+            unsigned long long m = 0;
+            for (int j = 0; j < a.k; ++j) {
+                const int p = pp[tl * a.k + j];
+                if (p >= 0) m |= 1ull << (p / epr);
+            }
+            uint8_t *row = a.in_rank + (size_t)(t0 + tl) * a.R;
+            for (int r = 0; r < a.R; ++r) row[r] = (uint8_t)((m >> r) & 1ull);
+            while (m) {
+                atomicAdd(&tokr[__ffsll((long long)m) - 1], 1);
+                m &= m - 1;
+            }
         }
-        a.in_rank[(size_t)(t0 + tl) * a.R + r] = (uint8_t)hit;
-        if (hit) atomicAdd(&tokr[r], 1);
+    } else {
+        for (int i = threadIdx.x; i < nt * a.R; i += blockDim.x) {
+            const int tl = i / a.R, r = i - tl * a.R;
+            int hit = 0;
+            for (int j = 0; j < a.k; ++j) {
+                const int p = pp[tl * a.k + j];
+                hit |= (p >= 0 && p / epr == r);
+            }
+            a.in_rank[(size_t)(t0 + tl) * a.R + r] = (uint8_t)hit;
+            if (hit) atomicAdd(&tokr[r], 1);
+        }
     }
     __syncthreads();
 
