@@ -15,6 +15,11 @@ namespace ep {
 
 namespace {
 
+// shared memory of the last block: the count / slot phase tables, then a
+// copy of the pair list (count writes it at P + R, slot keeps its own there)
+#define SMALL_SMEM_PAIRS_OFFSET(a) \
+    (2 * (a).P + 1 + (a).hist_warps * (a).P + (a).T * (a).k)
+
 template <int EPL>
 __global__ void __launch_bounds__(256)
 route_layout_small_kernel(RouteArgs r, LayoutArgs a, int vec4, int *done)
@@ -38,9 +43,14 @@ route_layout_small_kernel(RouteArgs r, LayoutArgs a, int vec4, int *done)
     __syncthreads();
     if (!is_last) return;
     __threadfence();  // every other block's top-k is visible to the last block
+    // the whole batch is tile 0; the slot phase reuses the pair list the
+    // count phase built, copied out of its way first
+    int *pairs = smem + SMALL_SMEM_PAIRS_OFFSET(a);
     layout_impl::count_tile(a, 0, smem, &bad_sh);
+    const int npairs = a.T * a.k;
+    for (int i = threadIdx.x; i < npairs; i += blockDim.x) pairs[i] = smem[a.P + a.R + i];
     __syncthreads();
-    layout_impl::slot_tile<256, true>(a, 0, smem, warp_tot);
+    layout_impl::slot_tile<256, true>(a, 0, smem, warp_tot, pairs);
 }
 
 template <int EPL>
@@ -74,7 +84,8 @@ cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *don
     const size_t pairs = (size_t)r.T * r.k;
     const size_t count_ints = (size_t)a.P + a.R + pairs;
     const size_t slot_ints = (size_t)2 * a.P + 1 + (size_t)a.hist_warps * a.P + pairs;
-    const size_t smem = sizeof(int) * (count_ints > slot_ints ? count_ints : slot_ints);
+    // tables of the larger phase, then the copied pair list
+    const size_t smem = sizeof(int) * ((count_ints > slot_ints ? count_ints : slot_ints) + pairs);
     const int vec4 = (r.E % 4 == 0) && ((reinterpret_cast<uintptr_t>(r.logits) & 15) == 0);
     if (r.E <= 32) return launch_small<1>(r, a, vec4, done, smem, s);
     if (r.E <= 64) return launch_small<2>(r, a, vec4, done, smem, s);

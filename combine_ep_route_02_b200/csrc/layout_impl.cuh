@@ -12,9 +12,10 @@ namespace layout_impl {
 constexpr int BAD_EXPERT = 1;
 constexpr int BAD_REPLICA = 2;
 
-EP_DEV int phys_expert(const LayoutArgs &a, int t, int j, int &bad)
+// physical expert of logical expert e for token t; -1 (and a status bit)
+// when invalid
+EP_DEV int phys_of_id(const LayoutArgs &a, int t, int e, int &bad)
 {
-    const int e = a.topk_idx[(size_t)t * a.k + j];
     if ((unsigned)e >= (unsigned)a.E) {
         bad |= BAD_EXPERT;
         return -1;
@@ -31,6 +32,32 @@ EP_DEV int phys_expert(const LayoutArgs &a, int t, int j, int &bad)
         return -1;
     }
     return p;
+}
+
+// Fills pp[0..npairs) with the physical experts of the tile's pairs (and
+// counts them in hist when given).  Each thread issues the loads of up to
+// eight of its pairs before using any, so a tile costs few L2 round trips.
+EP_DEV void fill_pairs(const LayoutArgs &a, int t0, int npairs, int *pp, int *hist, int &bad)
+{
+    constexpr int U = 8;
+    const int32_t *ids = a.topk_idx + (size_t)t0 * a.k;
+    for (int i0 = threadIdx.x; i0 < npairs; i0 += U * blockDim.x) {
+        int e[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * (int)blockDim.x;
+            e[u] = (i < npairs) ? ids[i] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * (int)blockDim.x;
+            if (i < npairs) {
+                const int p = phys_of_id(a, t0 + i / a.k, e[u], bad);
+                pp[i] = p;
+                if (hist != nullptr && p >= 0) atomicAdd(&hist[p], 1);
+            }
+        }
+    }
 }
 
 // Counts one tile (the block's threads cooperate; smem: P + R + tile_tokens*k
@@ -52,11 +79,7 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
     __syncthreads();
 
     int bad = 0;
-    for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
-        const int p = phys_expert(a, t0 + i / a.k, i % a.k, bad);
-        pp[i] = p;
-        if (p >= 0) atomicAdd(&hist[p], 1);
-    }
+    fill_pairs(a, t0, npairs, pp, hist, bad);
     if (bad) atomicOr(&bad_sh, bad);
     __syncthreads();
 
@@ -135,7 +158,8 @@ EP_DEV int block_exclusive_scan(int *v, int n, int *warp_tot)
 // and are summed here; otherwise tile_cnt already holds exclusive per-tile
 // offsets and cnt_expert the totals.
 template <int NTHREADS, bool FUSED>
-EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot)
+EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
+                      const int *pp_ready = nullptr)
 {
     constexpr int NWARPS = NTHREADS / 32;
     const int HW = a.hist_warps;
@@ -193,8 +217,11 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot)
         }
     }
     int bad = 0;  // reported below from the count kernel's tile status words
-    for (int i = threadIdx.x; i < npairs; i += blockDim.x)
-        pp[i] = phys_expert(a, t0 + i / a.k, i % a.k, bad);
+    if (pp_ready != nullptr) {  // the same block counted this tile already
+        for (int i = threadIdx.x; i < npairs; i += blockDim.x) pp[i] = pp_ready[i];
+    } else {
+        fill_pairs(a, t0, npairs, pp, nullptr, bad);
+    }
     __syncthreads();
 
     if (tile == 0) {

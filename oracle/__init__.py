@@ -69,6 +69,10 @@ def lib() -> ctypes.CDLL:
         _lib.orc_bf16_encode.restype = U16
         _lib.orc_bf16_decode.argtypes = [U16]
         _lib.orc_bf16_decode.restype = F
+        _lib.orc_dispatch_backward.argtypes = [P, I, P, I, I, I, P]
+        _lib.orc_dispatch_backward.restype = None
+        _lib.orc_combine_backward.argtypes = [P, P, I, P, P, I, I, I, P, P]
+        _lib.orc_combine_backward.restype = None
         S = ctypes.c_size_t
         _lib.orc_e4m3_encode_array.argtypes = [P, S, P]
         _lib.orc_e4m3_encode_array.restype = None
@@ -211,3 +215,30 @@ def sigmoid_array(x):
     hard = np.zeros(a.shape, np.uint8)
     lib().orc_sigmoid_array(_ptr(a), a.size, _ptr(out), _ptr(hard))
     return out, hard
+
+
+def dispatch_backward(grad_recv, slot):
+    """grad_x bf16 bits (uint16 [T,H]) = sum_j grad_recv[slot[t,j]] (fp32, j order)."""
+    g = _np(grad_recv, np.uint16)
+    n, H = g.shape
+    sl = _np(slot, np.int32)
+    T, k = sl.shape
+    out = np.zeros((T, H), np.uint16)
+    lib().orc_dispatch_backward(_ptr(g), n, _ptr(sl), T, H, k, _ptr(out))
+    return out
+
+
+def combine_backward(grad_out, y, slot, topk_w):
+    """(grad_y bf16 bits uint16 [T*k,H] (untouched rows 0), grad_w fp32 [T,k])."""
+    g = _np(grad_out, np.uint16)
+    T, H = g.shape
+    ys = _np(y, np.uint16)
+    n = ys.shape[0]
+    sl = _np(slot, np.int32)
+    k = sl.shape[1]
+    w = _np(topk_w, np.float32)
+    gy = np.zeros((n, H), np.uint16)
+    gw = np.zeros((T, k), np.float32)
+    lib().orc_combine_backward(_ptr(g), _ptr(ys), n, _ptr(sl), _ptr(w), T, H, k, _ptr(gy),
+                               _ptr(gw))
+    return gy, gw

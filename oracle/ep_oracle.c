@@ -398,3 +398,61 @@ void orc_sigmoid_array(const float *x, size_t n, float *out, uint8_t *hard)
         hard[i] = (uint8_t)h;
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* backward (training): dispatch-backward and combine-backward        */
+/* ------------------------------------------------------------------ */
+/*
+ * DeepEP V2 summary, section "Usage for training, prefill and decoding":
+ * the backward of dispatch is a combine and the backward of combine is a
+ * dispatch.  Reading: the forward FP8 quantisation is treated as the
+ * identity (straight-through), so gradients travel in BF16.
+ *
+ * dispatch-backward: grad_x[t] = bf16( sum_j grad_recv[slot[t,j]] ), fp32
+ * accumulation in j order (the combine of R8 with unit weights).
+ */
+void orc_dispatch_backward(const uint16_t *grad_recv, int n_rows, const int32_t *slot,
+                           int T, int H, int k, uint16_t *grad_x)
+{
+    float *acc = malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) acc[h] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            int s = slot[(size_t)t * k + j];
+            if (s < 0 || s >= n_rows) continue;
+            const uint16_t *g = grad_recv + (size_t)s * H;
+            for (int h = 0; h < H; ++h) acc[h] = acc[h] + orc_bf16_decode(g[h]);
+        }
+        for (int h = 0; h < H; ++h) grad_x[(size_t)t * H + h] = orc_bf16_encode(acc[h]);
+    }
+    free(acc);
+}
+
+/*
+ * combine-backward, for out[t] = sum_j w[t,j] * y[slot[t,j]]:
+ *   grad_y[slot[t,j]] = bf16( fp32(w[t,j] * grad_out[t]) )   (rows of
+ *                        invalid slots are not written)
+ *   grad_w[t,j]       = sum_h grad_out[t,h] * y[slot[t,j],h], evaluated in
+ *                        fp64 and rounded once to fp32 (0 for invalid slots)
+ */
+void orc_combine_backward(const uint16_t *grad_out, const uint16_t *y, int n_rows,
+                          const int32_t *slot, const float *w, int T, int H, int k,
+                          uint16_t *grad_y, float *grad_w)
+{
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *g = grad_out + (size_t)t * H;
+        for (int j = 0; j < k; ++j) {
+            int s = slot[(size_t)t * k + j];
+            if (s < 0 || s >= n_rows) { grad_w[(size_t)t * k + j] = 0.0f; continue; }
+            float wj = w[(size_t)t * k + j];
+            const uint16_t *yr = y + (size_t)s * H;
+            double dot = 0.0;
+            for (int h = 0; h < H; ++h) {
+                float gh = orc_bf16_decode(g[h]);
+                grad_y[(size_t)s * H + h] = orc_bf16_encode(wj * gh);
+                dot += (double)gh * (double)orc_bf16_decode(yr[h]);
+            }
+            grad_w[(size_t)t * k + j] = (float)dot;
+        }
+    }
+}

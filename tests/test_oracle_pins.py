@@ -506,3 +506,63 @@ def test_identity_expert_round_trip():
     outb = oracle.combine(yb, lay["slot"], w)
     gotb = torch.from_numpy(outb.view(np.int16)).view(torch.bfloat16).float().numpy()
     assert (np.abs(gotb - x) <= 2.0 ** -8 * np.abs(x) + 1e-30).all()
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def _bf16f(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def test_dispatch_backward_is_the_adjoint_of_dispatch():
+    """<dispatch(x), r> == <x, dispatch_backward(r)> for the bf16 permutation
+    (up to the bf16 rounding of the backward sum)"""
+    rng = np.random.default_rng(31)
+    T, H, k = 50, 256, 4
+    x = _bf16_rows(rng, T, H)
+    r = _bf16_rows(rng, T * k, H)
+    slot = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    rx, _ = oracle.dispatch(x, slot, fp8=False)
+    lhs = float((_bf16f(rx) * r.double().numpy()).sum())
+    gx = oracle.dispatch_backward(r, slot)
+    rhs = float((x.double().numpy() * _bf16f(gx)).sum())
+    mag = float((np.abs(x.double().numpy()) * np.abs(_bf16f(gx))).sum())
+    assert abs(lhs - rhs) <= 2.0 ** -8 * mag
+    # exact restatement of the sum (fp64, then the bf16 rounding bound)
+    ref = r.double().numpy()[slot].sum(axis=1)
+    assert (np.abs(_bf16f(gx) - ref) <= 2.0 ** -8 * np.abs(ref) + k * 2.0 ** -23 *
+            np.abs(r.double().numpy()[slot]).sum(axis=1) + 1e-30).all()
+
+
+def test_combine_backward_gradients():
+    rng = np.random.default_rng(32)
+    T, H, k = 40, 384, 6
+    y = _bf16_rows(rng, T * k, H)
+    g = _bf16_rows(rng, T, H)
+    slot = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    w = rng.uniform(0.05, 1.5, (T, k)).astype(np.float32)
+    gy, gw = oracle.combine_backward(g, y, slot, w)
+    gf, yf = g.double().numpy(), y.double().numpy()
+    # grad_w: derivative of sum_h g[t,h] * out[t,h] wrt w[t,j] is <g[t], y[slot]>
+    ref_w = np.einsum("th,tjh->tj", gf, yf[slot])
+    assert np.allclose(gw, ref_w, rtol=1e-6, atol=1e-6)
+    # grad_y rows: w * g[t], one fp32 product rounded to bf16
+    for t in range(T):
+        for j in range(k):
+            exp = torch.from_numpy((w[t, j] * g[t].float().numpy()).astype(np.float32)).to(
+                torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(gy[slot[t, j]], exp)
+    # adjoint: <combine(y), g> == <y, grad_y> (before bf16 rounding of either side)
+    out = oracle.combine(y, slot, w)
+    lhs = float((_bf16f(out) * gf).sum())
+    rhs = float((yf * _bf16f(gy)).sum())
+    assert abs(lhs - rhs) <= 2.0 ** -7 * float((np.abs(_bf16f(out)) * np.abs(gf)).sum())
+    # a finite-difference check of one weight's gradient
+    t, j, eps = 3, 2, 1e-3
+    w2 = w.copy()
+    w2[t, j] += eps
+    f = lambda ww: (np.einsum("tj,tjh->th", ww.astype(np.float64), yf[slot]) * gf).sum()
+    delta = float(w2[t, j]) - float(w[t, j])  # the step actually stored in fp32
+    assert (f(w2) - f(w)) / delta == pytest.approx(gw[t, j], rel=1e-6, abs=1e-6)
