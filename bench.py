@@ -247,6 +247,8 @@ def main():
                     help="run the workload with this many tokens instead (small cases for "
                          "profiler captures); 0 = the workload's own T")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the training backward (dispatch/combine backward)")
     args = ap.parse_args()
     faulthandler.enable()
     cfg = CONFIGS[args.config]
@@ -395,6 +397,45 @@ def main():
         mb.check_status()
         micro_ms = reduce_max(m0.elapsed_time(m1), dist, "cuda")
         del mb
+    # backward pass of the training step (dispatch-backward = combine of the
+    # gradient rows, combine-backward = scaled scatter + weight gradients),
+    # events around each call on the launching stream
+    backward = None
+    if not args.no_backward:
+        from combine_ep_route_02_b200 import ep_combine_backward, ep_dispatch_backward
+        g_out = device_normal_bf16(cfg.T, cfg.H, seed=100 + rank)
+        g_x = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+        g_y = torch.empty((cfg.T * cfg.topk, cfg.H), dtype=torch.bfloat16, device="cuda")
+        g_w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+        Kb = max(3, min(K, 50))
+        b0, b1, b2 = (events()[:Kb] for _ in range(3))
+        for i in range(args.warmup + Kb):
+            j = i - args.warmup
+            if flush:
+                flush_l2(i)
+            if j >= 0:
+                b0[j].record(stream)
+            ep_dispatch_backward(y, path.slot, cfg.T, cfg.H, cfg.topk, g_x,
+                                 dev_status=path.copy_status)
+            if j >= 0:
+                b1[j].record(stream)
+            ep_combine_backward(g_out, y, path.slot, path.topk_w, cfg.T, cfg.H, cfg.topk, g_y, g_w,
+                                dev_status=path.copy_status)
+            if j >= 0:
+                b2[j].record(stream)
+        torch.cuda.synchronize()
+        path.check_status()
+        db_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(b0, b1))
+        cb_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(b1, b2))
+        T_, H_, k_ = cfg.T, cfg.H, cfg.topk
+        db_bytes = T_ * k_ * 2 * H_ + T_ * 2 * H_ + T_ * k_ * 4
+        cb_bytes = T_ * 2 * H_ + 2 * T_ * k_ * 2 * H_ + T_ * k_ * 12
+        backward = {"dispatch_backward_us": db_ms * 1e3,
+                    "dispatch_backward_gbs": db_bytes / (db_ms * 1e-3) / 1e9,
+                    "combine_backward_us": cb_ms * 1e3,
+                    "combine_backward_gbs": cb_bytes / (cb_ms * 1e-3) / 1e9,
+                    "tokens_per_s": T_ * world / ((db_ms + cb_ms) * 1e-3)}
+        del g_out, g_x, g_y, g_w
     t_wall1 = time.perf_counter()
     sampler.stop()
     tot_ms = micro_ms if micro_ms is not None else seq_ms
@@ -497,6 +538,7 @@ def main():
             "roofline": roofline,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "backward": backward,
             "clocks": sampler.summary(t_wall0, t_wall1),
             "wall_s_timed": t_wall1 - t_wall0,
             **extra,

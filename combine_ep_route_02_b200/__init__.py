@@ -19,6 +19,8 @@ from ._binding import (  # noqa: F401
     EpError,
     RouteCfg,
     ep_combine,
+    ep_combine_backward,
+    ep_dispatch_backward,
     ep_dispatch,
     ep_dispatch_layout,
     ep_route,

@@ -27,7 +27,8 @@ EP_DEV_TIMEOUT = 4
 
 # every symbol declared in include/ep.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
-           "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout")
+           "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout",
+           "ep_dispatch_backward", "ep_combine_backward")
 
 
 class EpError(RuntimeError):
@@ -70,6 +71,10 @@ def lib() -> ctypes.CDLL:
         L.ep_route_layout.argtypes = [P, P, I, RouteCfg, I, I, P, P, I,
                                       P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.ep_route_layout.restype = I
+        L.ep_dispatch_backward.argtypes = [P, P, I, I, I, P, I, P, P]
+        L.ep_dispatch_backward.restype = I
+        L.ep_combine_backward.argtypes = [P, P, P, P, I, I, I, P, P, I, P, P]
+        L.ep_combine_backward.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -149,3 +154,17 @@ def ep_route_layout(logits, bias, T, cfg: RouteCfg, P, R, phys_of, n_rep, max_re
         _ptr(topk_idx), _ptr(topk_w), _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank),
         _ptr(rank_off), _ptr(tok_rank), _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace),
         _ptr(dev_status), _stream(stream)))
+
+
+def ep_dispatch_backward(grad_recv, slot, T, H, k, grad_x, num_sms=0, dev_status=None,
+                         stream=None):
+    _check("ep_dispatch_backward", lib().ep_dispatch_backward(
+        _ptr(grad_recv), _ptr(slot), T, H, k, _ptr(grad_x), num_sms, _ptr(dev_status),
+        _stream(stream)))
+
+
+def ep_combine_backward(grad_out, y, slot, topk_w, T, H, k, grad_y, grad_w, num_sms=0,
+                        dev_status=None, stream=None):
+    _check("ep_combine_backward", lib().ep_combine_backward(
+        _ptr(grad_out), _ptr(y), _ptr(slot), _ptr(topk_w), T, H, k, _ptr(grad_y), _ptr(grad_w),
+        num_sms, _ptr(dev_status), _stream(stream)))

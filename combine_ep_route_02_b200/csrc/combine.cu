@@ -44,7 +44,9 @@ combine_kernel(const uint16_t *__restrict__ y, const int32_t *__restrict__ slot,
                 const int j = j0 + u;
                 const int s = (j < k) ? __ldg(slot + (size_t)t * k + j) : -1;
                 ok[u] = (unsigned)s < (unsigned)n_rows;
-                wj[u] = ok[u] ? __ldg(w + (size_t)t * k + j) : 0.0f;
+                // w == nullptr: unit weights (the dispatch backward); the
+                // product by 1 is exact, so the sum is the plain fp32 sum
+                wj[u] = ok[u] ? (w != nullptr ? __ldg(w + (size_t)t * k + j) : 1.0f) : 0.0f;
                 v[u] = ok[u] ? ld_stream(y + (size_t)s * H + (size_t)c * 8) : make_uint4(0, 0, 0, 0);
             }
             // fp32 accumulation in j order: acc = RN(acc + RN(w * y)); the

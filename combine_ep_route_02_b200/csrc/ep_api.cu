@@ -237,4 +237,46 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
     return from_cuda(launch_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, int T, int H,
+                               int k, void *grad_x_bf16, int num_sms, int32_t *dev_status,
+                               ep_stream_t stream)
+{
+    if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
+    if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!grad_recv_bf16 || !slot || !grad_x_bf16)) return EP_ERR_INVALID;
+    if (!aligned(grad_recv_bf16, 16) || !aligned(grad_x_bf16, 16) || !aligned(slot, 4) ||
+        !aligned(dev_status, 4))
+        return EP_ERR_INVALID;
+    CombineArgs a{grad_recv_bf16, slot, nullptr, T, H, k, grad_x_bf16,
+                  streaming_grid(num_sms, cached_blocks_per_sm(2))};
+    return from_cuda(launch_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, const int32_t *slot,
+                              const float *topk_w, int T, int H, int k, void *grad_y_bf16,
+                              float *grad_w, int num_sms, int32_t *dev_status,
+                              ep_stream_t stream)
+{
+    if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
+    if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!grad_out_bf16 || !y_bf16 || !slot || !topk_w || !grad_y_bf16 || !grad_w))
+        return EP_ERR_INVALID;
+    if (!aligned(grad_out_bf16, 16) || !aligned(y_bf16, 16) || !aligned(grad_y_bf16, 16) ||
+        !aligned(slot, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4) || !aligned(dev_status, 4))
+        return EP_ERR_INVALID;
+    static volatile int occ[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int per_sm = dev < 64 ? occ[dev] : 0;
+    if (per_sm <= 0) {
+        per_sm = combine_backward_blocks_per_sm();
+        if (dev < 64) occ[dev] = per_sm;
+    }
+    CombineBackwardArgs a{grad_out_bf16, y_bf16, slot, topk_w, T, H, k, grad_y_bf16, grad_w,
+                          streaming_grid(num_sms, per_sm)};
+    return from_cuda(launch_combine_backward(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

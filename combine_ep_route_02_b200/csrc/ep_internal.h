@@ -99,6 +99,17 @@ inline int layout_tiles(int T, int k, int P)
     const int tt = layout_tile_tokens(T, k, P);
     return (T + tt - 1) / tt;
 }
+struct CombineBackwardArgs {
+    const void *g;     // grad_out bf16 [T, H]
+    const void *y;     // expert rows bf16 [T*k, H]
+    const int32_t *slot;
+    const float *w;
+    int T, H, k;
+    void *grad_y;      // bf16 [T*k, H]
+    float *grad_w;     // [T, k]
+    int grid;
+};
+
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 // workspace bytes: tile_cnt, tile_tok, tile_bad, each 256-byte aligned, then
 // 256 bytes holding the fused small-batch kernel's completion counter
@@ -146,6 +157,8 @@ cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *don
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_combine_backward(const CombineBackwardArgs &a, cudaStream_t s);
+int combine_backward_blocks_per_sm();
 
 // resident blocks per SM for each streaming kernel at its block size
 int dispatch_blocks_per_sm(int fp8);

@@ -242,6 +242,35 @@ ep_status ep_dispatch_layout_noalloc(const int32_t *topk_idx, int T, int k, int 
                                      uint8_t *in_rank, int32_t *slot, int32_t *src,
                                      int32_t *dev_status, ep_stream_t stream);
 
+/*
+ * Backward of dispatch (training): the DeepEP V2 summary (section "Usage for
+ * training, prefill and decoding") notes that dispatch's backward is a
+ * combine.  grad_x[t] = bf16( sum_j grad_recv[slot[t,j]] ), fp32 in j order:
+ * ep_combine with unit weights.  With an FP8 forward dispatch the
+ * quantisation is treated as the identity; gradients travel in BF16.
+ *   grad_recv_bf16  bf16 [T*k, H] gradients of the receive rows
+ *   grad_x_bf16     bf16 [T, H] (out)
+ * Alignment, slot handling and dev_status as for ep_combine.
+ */
+ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, int T, int H,
+                               int k, void *grad_x_bf16, int num_sms, int32_t *dev_status,
+                               ep_stream_t stream);
+
+/*
+ * Backward of combine (training): combine's backward is a dispatch (same
+ * section).  For out[t] = sum_j w[t,j] y[slot[t,j]]:
+ *   grad_y[slot[t,j]] = bf16( fp32(w[t,j] * grad_out[t]) )   bf16 [T*k, H]
+ *   grad_w[t,j]       = sum_h grad_out[t,h] * y[slot[t,j],h]  fp32 [T, k]
+ * The dot products are accumulated in fp32 in an unspecified order (within
+ * about 1e-5 of the sum of |terms| of the exact value).  Rows of invalid
+ * slots are not written and their grad_w is 0.  16-byte alignment for the
+ * bf16 arrays; dev_status as for ep_combine.
+ */
+ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, const int32_t *slot,
+                              const float *topk_w, int T, int H, int k, void *grad_y_bf16,
+                              float *grad_w, int num_sms, int32_t *dev_status,
+                              ep_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *ep_status_string(ep_status status);
 

@@ -552,3 +552,53 @@ def test_route_layout_fused_equals_two_calls(name, T):
     b.route_layout(lg, bs)
     torch.cuda.synchronize()
     assert torch.equal(a.slot, b.slot)
+
+
+# ---------------------------------------------------------------------------
+# backward (training)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["v3", "ds16b", "tiny"])
+def test_dispatch_backward(name):
+    from combine_ep_route_02_b200 import ep_dispatch_backward
+    cfg = CONFIGS[name]
+    wl = workload(name)
+    idx, _, _ = oracle_route(cfg, wl)
+    slot = oracle_layout(cfg, wl, idx)["slot"].copy()
+    slot[1, 0] = -1
+    g = device_normal_bf16(cfg.T * cfg.topk, cfg.H, seed=7)
+    gx = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    ep_dispatch_backward(g, torch.from_numpy(slot).cuda(), cfg.T, cfg.H, cfg.topk, gx)
+    torch.cuda.synchronize()
+    ref = oracle.dispatch_backward(g.cpu(), slot)
+    assert_combine_close(u16(gx), ref)
+    assert np.array_equal(u16(gx), ref)
+
+
+@pytest.mark.parametrize("name", ["v3", "ds16b", "skew"])
+def test_combine_backward(name):
+    from combine_ep_route_02_b200 import ep_combine_backward
+    cfg = CONFIGS[name] if name != "skew" else CONFIGS[name].scaled(2000)
+    wl = workload(name) if name != "skew" else Workload(cfg, seed=3)
+    idx, w, _ = oracle_route(cfg, wl)
+    slot = oracle_layout(cfg, wl, idx)["slot"].copy()
+    slot[2, 3] = -1
+    n = cfg.T * cfg.topk
+    y = device_normal_bf16(n, cfg.H, seed=8)
+    g = device_normal_bf16(cfg.T, cfg.H, seed=9)
+    gy = torch.zeros((n, cfg.H), dtype=torch.bfloat16, device="cuda")
+    gw = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    ep_combine_backward(g, y, torch.from_numpy(slot).cuda(), torch.from_numpy(w).cuda(), cfg.T,
+                        cfg.H, cfg.topk, gy, gw)
+    torch.cuda.synchronize()
+    ref_y, ref_w = oracle.combine_backward(g.cpu(), y.cpu(), slot, w)
+    assert np.array_equal(u16(gy), ref_y)
+    # fp32 dot products in a different order than the oracle's fp64 sum
+    yc, gc = y.cpu().double().numpy(), g.cpu().double().numpy()
+    valid = slot >= 0
+    mag = np.zeros_like(ref_w, dtype=np.float64)
+    mag[valid] = np.einsum("th,th->t", np.abs(gc)[np.nonzero(valid)[0]],
+                           np.abs(yc[slot[valid]]))
+    err = np.abs(gw.cpu().numpy().astype(np.float64) - ref_w)
+    assert (err <= 1e-5 * mag + 1e-6).all(), float((err - 1e-5 * mag).max())
+    assert (gw.cpu().numpy()[~valid] == 0).all()
