@@ -240,6 +240,9 @@ def main():
                          "overlap dispatch+combine of batch i); sequential: one step after "
                          "the other on one stream")
     ap.add_argument("--num-sms", type=int, default=0)
+    ap.add_argument("--split-sms", default="",
+                    help="micro-batch schedule: 'd,c' runs dispatch of batch i+1 on d SMs next "
+                         "to combine of batch i on c SMs; empty = one after the other")
     ap.add_argument("--ref-tokens", type=int, default=512,
                     help="tokens per oracle step (--impl reference and cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -383,7 +386,11 @@ def main():
             return _EpPath(cfg.T, cfg.H, cfg.E, cfg.n_group, cfg.topk_group, cfg.topk,
                            cfg.routed_scale, cfg.renorm, cfg.R, cfg.fp8, phys_of=wl.phys_of,
                            n_rep=wl.n_rep, num_sms=args.num_sms)
-        mb = EpMicroBatchPipeline(make_path)
+        split = None
+        if args.split_sms:
+            d_sms, c_sms = (int(v) for v in args.split_sms.split(","))
+            split = (d_sms, c_sms)
+        mb = EpMicroBatchPipeline(make_path, split_sms=split)
         mb.run([x] * args.warmup, [lg] * args.warmup, [bias] * args.warmup, [y] * args.warmup)
         torch.cuda.synchronize()
         barrier()
@@ -391,7 +398,7 @@ def main():
         m1 = torch.cuda.Event(enable_timing=True)
         m0.record(mb.s_route)
         mb.run([x] * K, [lg] * K, [bias] * K, [y] * K)
-        m1.record(mb.s_move)
+        m1.record(mb.s_last)
         torch.cuda.synchronize()
         barrier()
         mb.check_status()

@@ -92,6 +92,12 @@ EP_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
                  : "memory");
 }
 
+// plain arrive (count 1) on a CTA-local mbarrier
+EP_DEV void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Polls the barrier phase at most `limit` times; false if it never completed.
 EP_DEV bool mbar_wait(uint32_t bar, uint32_t phase, uint32_t limit)
 {

@@ -32,7 +32,9 @@ class EpPath:
         dev = torch.device(device)
         self.T, self.H, self.k, self.E, self.R = T, H, topk, num_experts, R
         self.fp8 = bool(fp8)
-        self.num_sms = num_sms
+        self.num_sms = num_sms          # SMs for dispatch and combine (0 = all)
+        self.dispatch_sms = num_sms
+        self.combine_sms = num_sms
         self.cfg = B.RouteCfg(num_experts, n_group, topk_group, topk, float(routed_scale),
                               int(bool(renorm)))
         if phys_of is not None:
@@ -89,12 +91,12 @@ class EpPath:
 
     def dispatch(self, x: torch.Tensor, stream=None):
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
-                      self.recv_scale, self.num_sms, self.copy_status, stream)
+                      self.recv_scale, self.dispatch_sms, self.copy_status, stream)
 
     def combine(self, y: torch.Tensor, stream=None, out: Optional[torch.Tensor] = None):
         out = self.out if out is None else out
         B.ep_combine(y, self.slot, self.topk_w, self.T, self.H, self.k, out,
-                     self.num_sms, self.copy_status, stream)
+                     self.combine_sms, self.copy_status, stream)
         return out
 
     def step(self, x, logits, bias, y, stream=None, out=None):
@@ -183,25 +185,41 @@ class EpHostPipeline:
 
 class EpMicroBatchPipeline:
     """Two micro-batches in flight, as in the two-micro-batch overlap of
-    DeepSeek's and Perplexity's EP deployments: routing and layout of batch
-    i+1 (arithmetic- and latency-bound) run on one stream while dispatch and
-    combine of batch i (HBM-bound) run on another.  Each of the two
+    DeepSeek's and Perplexity's EP deployments.
+
+    Routing and layout (arithmetic- and latency-bound) run on one stream.
+    With ``split_sms=None`` dispatch and combine of a batch follow each other
+    on a second stream, overlapping the next batch's routing.  With
+    ``split_sms=(d, c)`` they get a stream each and are capped to d and c SMs,
+    so the write-heavy dispatch of batch i+1 runs next to the read-heavy
+    combine of batch i and HBM sees a mix of reads and writes instead of a
+    pure write phase followed by a pure read phase.  Each of the two
     ``EpPath`` buffer sets serves every other batch; batch i+2 starts its
     routing only after batch i has finished its combine.
     """
 
-    def __init__(self, make_path, device="cuda"):
+    def __init__(self, make_path, device="cuda", split_sms=None):
         dev = torch.device(device)
         self.paths = [make_path(), make_path()]
+        self.split = split_sms
+        if split_sms is not None:
+            for p in self.paths:
+                p.dispatch_sms, p.combine_sms = split_sms
         self.s_route = torch.cuda.Stream(dev)
-        self.s_move = torch.cuda.Stream(dev)
-        self.layout_done = [torch.cuda.Event() for _ in range(2)]
-        self.move_done = [torch.cuda.Event() for _ in range(2)]
+        self.s_move = torch.cuda.Stream(dev)     # dispatch (and combine unless split)
+        self.s_comb = torch.cuda.Stream(dev) if split_sms is not None else self.s_move
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.layout_done, self.disp_done, self.move_done = ev(), ev(), ev()
+
+    @property
+    def s_last(self):
+        """the stream that carries the last combine"""
+        return self.s_comb
 
     def run(self, xs, logits, biases, ys):
         """Enqueues batch i = (xs[i], logits[i], biases[i], expert outputs
         ys[i]); results land in ``self.paths[i % 2].out``.  Returns without
-        synchronising; ``self.s_move`` carries the last combine."""
+        synchronising; ``self.s_last`` carries the last combine."""
         for i in range(len(xs)):
             b = i & 1
             p = self.paths[b]
@@ -213,8 +231,11 @@ class EpMicroBatchPipeline:
             self.s_move.wait_event(self.layout_done[b])
             with torch.cuda.stream(self.s_move):
                 p.dispatch(xs[i], stream=self.s_move)
-                p.combine(ys[i], stream=self.s_move)
-                self.move_done[b].record(self.s_move)
+                self.disp_done[b].record(self.s_move)
+            self.s_comb.wait_event(self.disp_done[b])
+            with torch.cuda.stream(self.s_comb):
+                p.combine(ys[i], stream=self.s_comb)
+                self.move_done[b].record(self.s_comb)
 
     def check_status(self):
         for p in self.paths:
