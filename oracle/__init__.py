@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_route.restype = None
         _lib.orc_layout.argtypes = [P, I, I, I, I, I, P, P, I, P, P, P, P, P, P, P, P]
         _lib.orc_layout.restype = I
+        _lib.orc_layout_aligned.argtypes = [P, I, I, I, I, I, P, P, I, I, P, P, P, P, P, P, P, P]
+        _lib.orc_layout_aligned.restype = I
         _lib.orc_dispatch.argtypes = [P, I, I, I, P, I, I, P, P]
         _lib.orc_dispatch.restype = None
         _lib.orc_quantize_row.argtypes = [P, I, P, P]
@@ -123,22 +125,27 @@ def route(logits, bias, n_group: int, topk_group: int, topk: int,
     return idx, w, hard
 
 
-def layout(topk_idx, E: int, P: int, R: int, phys_of=None, n_rep=None):
-    """Dispatch layout.  Returns a dict of arrays plus ``status`` bits."""
+def layout(topk_idx, E: int, P: int, R: int, phys_of=None, n_rep=None, row_align: int = 1):
+    """Dispatch layout (expert starts padded to row_align rows when > 1).
+    Returns a dict of arrays plus ``status`` bits; ``src`` has one entry per
+    receive row (padding rows -1)."""
     ti = _np(topk_idx, np.int32)
     T, k = ti.shape
     po = _np(phys_of, np.int32)
     nr = _np(n_rep, np.int32)
     max_rep = 0 if po is None else po.shape[1]
+    n_src = T * k + P * (row_align - 1)
     out = dict(
         cnt_expert=np.zeros(P, np.int32), expert_off=np.zeros(P + 1, np.int32),
         rows_rank=np.zeros(R, np.int32), rank_off=np.zeros(R + 1, np.int32),
         tok_rank=np.zeros(R, np.int32), in_rank=np.zeros((T, R), np.uint8),
-        slot=np.zeros((T, k), np.int32), src=np.full(T * k, -1, np.int32))
-    st = lib().orc_layout(_ptr(ti), T, k, E, P, R, _ptr(po), _ptr(nr), max_rep,
-                          *(_ptr(out[n]) for n in ("cnt_expert", "expert_off", "rows_rank",
-                                                   "rank_off", "tok_rank", "in_rank",
-                                                   "slot", "src")))
+        slot=np.zeros((T, k), np.int32), src=np.full(n_src, -1, np.int32))
+    st = lib().orc_layout_aligned(_ptr(ti), T, k, E, P, R, _ptr(po), _ptr(nr), max_rep,
+                                  row_align,
+                                  *(_ptr(out[n]) for n in ("cnt_expert", "expert_off",
+                                                           "rows_rank", "rank_off", "tok_rank",
+                                                           "in_rank", "slot", "src")))
+    out["src"] = out["src"][:int(out["expert_off"][P])]
     out["status"] = int(st)
     return out
 

@@ -220,6 +220,12 @@ void orc_route(const float *logits, const float *bias, int T, int E,
 /* dispatch layout                                                     */
 /* ------------------------------------------------------------------ */
 
+int orc_layout_aligned(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       int row_align, int32_t *cnt_expert, int32_t *expert_off,
+                       int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                       uint8_t *in_rank, int32_t *slot, int32_t *src);
+
 /* physical expert of pair (t, j); -1 (and a status bit) when invalid */
 static int phys_expert(const int32_t *topk_idx, int t, int j, int k, int E, int P,
                        const int32_t *phys_of, const int32_t *n_rep, int max_rep,
@@ -247,6 +253,26 @@ int orc_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
                int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
                int32_t *slot, int32_t *src)
 {
+    return orc_layout_aligned(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, 1,
+                              cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
+                              in_rank, slot, src);
+}
+
+/*
+ * The same layout with every expert's first receive row a multiple of
+ * row_align (the row tile of a grouped GEMM consuming the receive buffer,
+ * the "GEMM layout" of the DeepEP V2 summary): expert p occupies rows
+ * [expert_off[p], expert_off[p] + cnt_expert[p]) followed by
+ * round_up(cnt, row_align) - cnt padding rows whose src is -1.
+ * expert_off, rows_rank and rank_off count padded rows; cnt_expert and
+ * tok_rank do not.  src has expert_off[P] entries.
+ */
+int orc_layout_aligned(const int32_t *topk_idx, int T, int k, int E, int P, int R,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       int row_align, int32_t *cnt_expert, int32_t *expert_off,
+                       int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                       uint8_t *in_rank, int32_t *slot, int32_t *src)
+{
     int status = 0;
     int epr = P / R;
     int32_t *fill = calloc((size_t)P, sizeof(int32_t));
@@ -259,7 +285,12 @@ int orc_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
         }
 
     expert_off[0] = 0;
-    for (int p = 0; p < P; ++p) expert_off[p + 1] = expert_off[p] + cnt_expert[p];
+    for (int p = 0; p < P; ++p) {
+        int padded = (cnt_expert[p] + row_align - 1) / row_align * row_align;
+        expert_off[p + 1] = expert_off[p] + padded;
+    }
+    for (int p = 0; p < P; ++p)
+        for (int r = expert_off[p] + cnt_expert[p]; r < expert_off[p + 1]; ++r) src[r] = -1;
 
     for (int t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {

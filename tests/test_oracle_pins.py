@@ -566,3 +566,37 @@ def test_combine_backward_gradients():
     f = lambda ww: (np.einsum("tj,tjh->th", ww.astype(np.float64), yf[slot]) * gf).sum()
     delta = float(w2[t, j]) - float(w[t, j])  # the step actually stored in fp32
     assert (f(w2) - f(w)) / delta == pytest.approx(gw[t, j], rel=1e-6, abs=1e-6)
+
+
+@pytest.mark.parametrize("align", [1, 4, 64, 128])
+def test_layout_row_alignment(align):
+    """padded expert starts: multiples of the row tile, the same rows per
+    expert in the same order, padding rows marked -1"""
+    cfg = CONFIGS["skew"].scaled(300)
+    wl = Workload(cfg, seed=5)
+    idx, _, _ = oracle.route(wl.logits, wl.bias, cfg.n_group, cfg.topk_group, cfg.topk,
+                             cfg.routed_scale, cfg.renorm)
+    po, nr = wl.phys_of.numpy(), wl.n_rep.numpy()
+    base = oracle.layout(idx, cfg.E, cfg.n_phys, cfg.R, po, nr)
+    lay = oracle.layout(idx, cfg.E, cfg.n_phys, cfg.R, po, nr, row_align=align)
+    P = cfg.n_phys
+    cnt = lay["cnt_expert"]
+    assert np.array_equal(cnt, base["cnt_expert"])
+    assert np.array_equal(lay["tok_rank"], base["tok_rank"])
+    assert np.array_equal(lay["in_rank"], base["in_rank"])
+    off = lay["expert_off"]
+    assert (off % align == 0).all()
+    assert np.array_equal(np.diff(off), -(-cnt // align) * align)
+    # pair (t, j) keeps its rank inside its expert
+    phys = np.searchsorted(base["expert_off"], base["slot"], side="right") - 1
+    assert np.array_equal(lay["slot"] - off[phys], base["slot"] - base["expert_off"][phys])
+    src = lay["src"]
+    assert src.size == off[P]
+    assert np.array_equal(src[lay["slot"].ravel()], np.arange(cfg.T * cfg.topk))
+    assert (src >= 0).sum() == cfg.T * cfg.topk
+    epr = P // cfg.R
+    assert np.array_equal(lay["rank_off"], off[::epr])
+    assert np.array_equal(lay["rows_rank"], np.diff(off[::epr]))
+    if align == 1:
+        for n in ("expert_off", "slot", "src", "rows_rank", "rank_off"):
+            assert np.array_equal(lay[n], base[n])
