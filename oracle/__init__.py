@@ -82,6 +82,14 @@ def lib() -> ctypes.CDLL:
         _lib.orc_bf16_encode_array.restype = None
         _lib.orc_sigmoid_array.argtypes = [P, S, P, P]
         _lib.orc_sigmoid_array.restype = None
+        _lib.orc_silu_bf16.argtypes = [U16, ctypes.POINTER(I)]
+        _lib.orc_silu_bf16.restype = U16
+        _lib.orc_silu_bf16_array.argtypes = [P, S, P, P]
+        _lib.orc_silu_mul_row.argtypes = [P, I, P]
+        _lib.orc_silu_mul_row.restype = None
+        _lib.orc_silu_mul_quant.argtypes = [P, I, I, P, P, I, I, P, P]
+        _lib.orc_silu_mul_quant.restype = None
+        _lib.orc_silu_bf16_array.restype = None
     return _lib
 
 
@@ -249,3 +257,33 @@ def combine_backward(grad_out, y, slot, topk_w):
     lib().orc_combine_backward(_ptr(g), _ptr(ys), n, _ptr(sl), _ptr(w), T, H, k, _ptr(gy),
                                _ptr(gw))
     return gy, gw
+
+
+def silu_bf16_array(g):
+    """(bf16 bits of silu(g) correctly rounded, hard flags) for bf16 bits g."""
+    a = _np(g, np.uint16)
+    out = np.zeros(a.shape, np.uint16)
+    hard = np.zeros(a.shape, np.uint8)
+    lib().orc_silu_bf16_array(_ptr(a), a.size, _ptr(out), _ptr(hard))
+    return out, hard
+
+
+def silu_mul_quant(gate_up, fp8: bool, expert_off=None, cnt_expert=None, act=None,
+                   act_scale=None):
+    """Expert activation of bf16 rows [n_rows, 2I] (uint16 bits).  Returns
+    (act, act_scale): e4m3 codes uint8 [n_rows, I] and fp32 [n_rows, I/128]
+    when fp8, else bf16 bits uint16 [n_rows, I] and None.  Only the rows the
+    counts select are written; pass act / act_scale to see the others kept."""
+    gu = _np(gate_up, np.uint16)
+    n, I2 = gu.shape
+    I = I2 // 2
+    if act is None:
+        act = np.zeros((n, I), np.uint8 if fp8 else np.uint16)
+    if fp8 and act_scale is None:
+        act_scale = np.zeros((n, max(I // 128, 1)), np.float32)
+    eo = _np(expert_off, np.int32)
+    ce = _np(cnt_expert, np.int32)
+    P = 0 if ce is None else ce.size
+    lib().orc_silu_mul_quant(_ptr(gu), n, I, _ptr(eo), _ptr(ce), P, int(bool(fp8)), _ptr(act),
+                             _ptr(act_scale) if fp8 else None)
+    return act, (act_scale if fp8 else None)

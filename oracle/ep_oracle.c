@@ -49,6 +49,18 @@
  *     scale 0 and all payload bytes 0x00.
  *  R8 combine: acc = 0; acc = fp32_RN(acc + fp32_RN(w_j * y_j)) in j order;
  *     out = bf16_RNE(acc).
+ *  R9 expert activation (SiLU, Perplexity blog section "Quantization"): the
+ *     first grouped GEMM's row holds [gate | up], I bf16 each (DeepSeek-V3's
+ *     gated SiLU expert).  s = bf16_RN(silu(g)), silu(g) = g / (1 + e^-g),
+ *     correctly rounded (fp64 evaluation; silu(-inf) = -0, silu(+inf) =
+ *     +inf); h = bf16_RN(fp32_RN(s * u)), as a BF16 model multiplies; then
+ *     h is quantised per 128 elements as in R7.
+ *  R10 GEMM layout: with a row tile A > 1, expert p's rows start at a
+ *     multiple of A and are followed by round_up(cnt, A) - cnt padding rows
+ *     (src = -1); expert_off / rank_off / rows_rank count padded rows.
+ *  R11 the activation reads the per-expert counts: it processes exactly the
+ *     rows [expert_off[p], expert_off[p] + cnt_expert[p]) and leaves padding
+ *     and unused rows untouched.
  */
 #include <math.h>
 #include <stdint.h>
@@ -486,4 +498,102 @@ void orc_combine_backward(const uint16_t *grad_out, const uint16_t *y, int n_row
             grad_w[(size_t)t * k + j] = (float)dot;
         }
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* expert activation: SiLU(gate) * up, then 1x128 FP8 (R9, R11)        */
+/* ------------------------------------------------------------------ */
+
+/* Round a finite double to bf16, to nearest, and flag values within 2^-44
+ * (relative) of a rounding midpoint.  bf16 keeps 8 significant bits down to
+ * 2^-126 and a fixed step of 2^-133 below.  An exact tie goes to the even
+ * neighbour, or, with tie_up set, to the neighbour toward +inf (for a value
+ * known to lie a hair above v). */
+static uint16_t bf16_round_double(double v, int *hard, int tie_up)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0x0000u;
+    double a = fabs(v);
+    if (hard) *hard = 0;
+    if (a == 0.0) return sign;
+    double q;
+    if (a < 0x1p-126) {
+        q = 0x1p-133;
+    } else {
+        int e;
+        frexp(a, &e);            /* 2^(e-1) <= a < 2^e */
+        q = ldexp(1.0, e - 1 - 7);
+    }
+    double n = a / q;            /* exact: a power-of-two scaling */
+    double r = round_half_even(n);
+    if (tie_up && n - floor(n) == 0.5) r = sign ? floor(n) : floor(n) + 1.0;
+    if (hard && !tie_up) *hard = fabs(n - floor(n) - 0.5) <= ldexp(n, -44);
+    double res = r * q;
+    if (res >= 0x1p128) return sign | 0x7F80u; /* rounds past the largest finite */
+    return sign | (uint16_t)(float_to_bits((float)res) >> 16); /* res is a bf16 value */
+}
+
+/* R9: SiLU of a bf16 value, correctly rounded to bf16. */
+uint16_t orc_silu_bf16(uint16_t g, int *hard)
+{
+    float gf = orc_bf16_decode(g);
+    if (hard) *hard = 0;
+    if (isnan(gf)) return (uint16_t)(g | 0x0040u);
+    if (isinf(gf)) return gf > 0 ? 0x7F80u : 0x8000u;
+    double x = (double)gf;
+    /* silu(x) - x/2 = x tanh(x/2) / 2 > 0 for x != 0.  For tiny x that
+     * difference is far below fp64 resolution, the fp64 quotient is x/2
+     * exactly, and x/2 can be a bf16 midpoint (odd multiples of 2^-134): the
+     * exact value lies just above it, so such a tie rounds toward +inf. */
+    if (fabs(x) < 0x1p-100) return bf16_round_double(x / 2.0, hard, 1);
+    return bf16_round_double(x / (1.0 + exp(-x)), hard, 0);
+}
+
+void orc_silu_bf16_array(const uint16_t *g, size_t n, uint16_t *out, uint8_t *hard)
+{
+    for (size_t i = 0; i < n; ++i) {
+        int h = 0;
+        out[i] = orc_silu_bf16(g[i], &h);
+        hard[i] = (uint8_t)h;
+    }
+}
+
+/* R9: h[i] = bf16(fp32(silu_bf16(gate[i]) * up[i])) for one row. */
+void orc_silu_mul_row(const uint16_t *gate_up, int I, uint16_t *h)
+{
+    for (int i = 0; i < I; ++i) {
+        float s = orc_bf16_decode(orc_silu_bf16(gate_up[i], NULL));
+        float u = orc_bf16_decode(gate_up[I + i]);
+        float prod = s * u;
+        h[i] = orc_bf16_encode(prod);
+    }
+}
+
+/*
+ * Expert activation over the receive rows (R9, R11).  gate_up bf16
+ * [n_rows, 2I]; expert_off / cnt_expert select the rows (NULL: every row).
+ * fp8: act is e4m3 [n_rows, I] and act_scale fp32 [n_rows, I/128];
+ * otherwise act is bf16 [n_rows, I] (h itself).  Rows outside the selection
+ * are not written.
+ */
+void orc_silu_mul_quant(const uint16_t *gate_up, int n_rows, int I, const int32_t *expert_off,
+                        const int32_t *cnt_expert, int P, int fp8, void *act, float *act_scale)
+{
+    uint16_t *h = malloc(sizeof(uint16_t) * (size_t)(I > 0 ? I : 1));
+    int S = I / 128;
+    int n_groups = expert_off ? P : 1;
+    for (int p = 0; p < n_groups; ++p) {
+        int r0 = expert_off ? expert_off[p] : 0;
+        int r1 = expert_off ? r0 + cnt_expert[p] : n_rows;
+        if (r1 > n_rows) r1 = n_rows;
+        for (int r = r0 < 0 ? 0 : r0; r < r1; ++r) {
+            const uint16_t *row = gate_up + (size_t)r * 2 * I;
+            if (fp8) {
+                orc_silu_mul_row(row, I, h);
+                orc_quantize_row(h, I, (uint8_t *)act + (size_t)r * I, act_scale + (size_t)r * S);
+            } else {
+                orc_silu_mul_row(row, I, (uint16_t *)act + (size_t)r * I);
+            }
+        }
+    }
+    free(h);
 }
