@@ -252,6 +252,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip timing the training backward (dispatch/combine backward)")
+    ap.add_argument("--no-gemm-layout", action="store_true",
+                    help="skip timing the GEMM layout (padded rows) and the expert activation")
+    ap.add_argument("--row-align", type=int, default=128,
+                    help="row tile of the GEMM layout timed after the step")
     args = ap.parse_args()
     faulthandler.enable()
     cfg = CONFIGS[args.config]
@@ -314,8 +318,8 @@ def main():
 
     K = args.steps
 
-    def events():
-        return [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    def events(n=None):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(K if n is None else n)]
 
     def total_ms(a, b):
         return reduce_max(sum(x.elapsed_time(y) for x, y in zip(a, b)), dist, "cuda")
@@ -415,7 +419,7 @@ def main():
         g_y = torch.empty((cfg.T * cfg.topk, cfg.H), dtype=torch.bfloat16, device="cuda")
         g_w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
         Kb = max(3, min(K, 50))
-        b0, b1, b2 = (events()[:Kb] for _ in range(3))
+        b0, b1, b2 = (events(Kb) for _ in range(3))
         for i in range(args.warmup + Kb):
             j = i - args.warmup
             if flush:
@@ -443,6 +447,53 @@ def main():
                     "combine_backward_gbs": cb_bytes / (cb_ms * 1e-3) / 1e9,
                     "tokens_per_s": T_ * world / ((db_ms + cb_ms) * 1e-3)}
         del g_out, g_x, g_y, g_w
+    # GEMM layout: expert rows padded to the grouped GEMM's row tile, and the
+    # expert activation silu(gate) * up -> e4m3 + 1x128 scales between the two
+    # expert GEMMs, over the rows the device-side counts select
+    gemm = None
+    if not args.no_gemm_layout:
+        A, I = args.row_align, cfg.inter
+        pa = EpPath(cfg.T, cfg.H, cfg.E, cfg.n_group, cfg.topk_group, cfg.topk,
+                    cfg.routed_scale, cfg.renorm, cfg.R, cfg.fp8, phys_of=wl.phys_of,
+                    n_rep=wl.n_rep, num_sms=args.num_sms, row_align=A)
+        gate_up = device_normal_bf16(pa.n_recv, 2 * I, seed=200 + rank)
+        act = torch.empty((pa.n_recv, I), dtype=torch.float8_e4m3fn, device="cuda")
+        act_sc = torch.empty((pa.n_recv, I // 128), dtype=torch.float32, device="cuda")
+        V = cfg.T * cfg.topk
+        act_bytes = V * (4 * I + I + 4 * (I // 128)) + pa.P * 8
+        act_flush = act_bytes < 2 * L2_BYTES
+        if act_flush and flush_w is None:
+            flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+            flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+        Ka = max(3, min(K, 50))
+        a0, a1, a2 = (events(Ka) for _ in range(3))
+        for i in range(args.warmup + Ka):
+            j = i - args.warmup
+            if act_flush:
+                flush_l2(i)
+            if j >= 0:
+                a0[j].record(stream)
+            pa.route_layout(lg, bias)
+            if j >= 0:
+                a1[j].record(stream)
+            pa.activation(gate_up, act, act_sc)
+            if j >= 0:
+                a2[j].record(stream)
+        torch.cuda.synchronize()
+        pa.check_status()
+        rl_a_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(a0, a1))
+        act_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(a1, a2))
+        used = int(pa.expert_off[-1].item())
+        act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
+        pk, pk_kind = peak_hbm()
+        gemm = {"row_align": A, "I": I, "recv_rows_capacity": pa.n_recv,
+                "recv_rows_used": used, "padding_rows": used - V,
+                "route_layout_us": rl_a_ms * 1e3,
+                "silu_mul_us": act_ms * 1e3, "silu_mul_gbs": act_gbs,
+                "silu_mul_frac": act_gbs / pk,
+                "silu_mul_bytes": act_bytes,
+                "l2": "flushed before each call" if act_flush else "inputs larger than L2"}
+        del pa, gate_up, act, act_sc
     t_wall1 = time.perf_counter()
     sampler.stop()
     tot_ms = micro_ms if micro_ms is not None else seq_ms
@@ -546,6 +597,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "backward": backward,
+            "gemm_layout": gemm,
             "clocks": sampler.summary(t_wall0, t_wall1),
             "wall_s_timed": t_wall1 - t_wall0,
             **extra,

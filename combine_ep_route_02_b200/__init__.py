@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     ep_dispatch_layout,
     ep_route,
     ep_route_layout,
+    ep_silu_mul,
     ep_workspace_size,
     lib,
 )

@@ -28,7 +28,7 @@ EP_DEV_TIMEOUT = 4
 # every symbol declared in include/ep.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
            "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout",
-           "ep_dispatch_backward", "ep_combine_backward")
+           "ep_dispatch_backward", "ep_combine_backward", "ep_silu_mul")
 
 
 class EpError(RuntimeError):
@@ -58,23 +58,25 @@ def lib() -> ctypes.CDLL:
         L.ep_workspace_size.restype = Z
         L.ep_route.argtypes = [P, P, I, RouteCfg, P, P, P]
         L.ep_route.restype = I
-        L.ep_dispatch_layout.argtypes = [P, I, I, I, I, I, P, P, I,
+        L.ep_dispatch_layout.argtypes = [P, I, I, I, I, I, P, P, I, I,
                                          P, P, P, P, P, P, P, P, P, P, P]
         L.ep_dispatch_layout.restype = I
-        L.ep_dispatch.argtypes = [P, I, I, I, P, I, P, P, I, P, P]
+        L.ep_dispatch.argtypes = [P, I, I, I, I, P, I, P, P, I, P, P]
         L.ep_dispatch.restype = I
-        L.ep_combine.argtypes = [P, P, P, I, I, I, P, I, P, P]
+        L.ep_combine.argtypes = [P, P, P, I, I, I, I, P, I, P, P]
         L.ep_combine.restype = I
         L.ep_dispatch_layout_noalloc.argtypes = [P, I, I, I, I, I, P, P, I,
                                                  P, P, P, P, P, P, P, P, P, P]
         L.ep_dispatch_layout_noalloc.restype = I
-        L.ep_route_layout.argtypes = [P, P, I, RouteCfg, I, I, P, P, I,
+        L.ep_route_layout.argtypes = [P, P, I, RouteCfg, I, I, P, P, I, I,
                                       P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.ep_route_layout.restype = I
-        L.ep_dispatch_backward.argtypes = [P, P, I, I, I, P, I, P, P]
+        L.ep_dispatch_backward.argtypes = [P, P, I, I, I, I, P, I, P, P]
         L.ep_dispatch_backward.restype = I
-        L.ep_combine_backward.argtypes = [P, P, P, P, I, I, I, P, P, I, P, P]
+        L.ep_combine_backward.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P, P]
         L.ep_combine_backward.restype = I
+        L.ep_silu_mul.argtypes = [P, I, I, P, P, I, I, P, P, I, P]
+        L.ep_silu_mul.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -113,23 +115,28 @@ def ep_route(logits, bias, T, cfg: RouteCfg, topk_idx, topk_w, stream=None):
 
 def ep_dispatch_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
                        expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
-                       workspace, dev_status, stream=None):
+                       workspace, dev_status, stream=None, *, row_align=1):
+    """row_align > 1: each expert's rows start on a multiple of row_align and
+    src needs T*k + P*(row_align-1) entries."""
     _check("ep_dispatch_layout", lib().ep_dispatch_layout(
-        _ptr(topk_idx), T, k, E, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
+        _ptr(topk_idx), T, k, E, P, R, _ptr(phys_of), _ptr(n_rep), max_rep, row_align,
         _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank), _ptr(rank_off), _ptr(tok_rank),
         _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace), _ptr(dev_status),
         _stream(stream)))
 
 
 def ep_dispatch(x, T, H, k, slot, fp8, recv_x, recv_scale, num_sms=0, dev_status=None,
-                stream=None):
-    _check("ep_dispatch", lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot), int(bool(fp8)),
-                                            _ptr(recv_x), _ptr(recv_scale), num_sms,
-                                            _ptr(dev_status), _stream(stream)))
+                stream=None, *, recv_rows=0):
+    """recv_rows: rows of recv_x (0 = T*k)."""
+    _check("ep_dispatch", lib().ep_dispatch(_ptr(x), T, H, k, recv_rows, _ptr(slot),
+                                            int(bool(fp8)), _ptr(recv_x), _ptr(recv_scale),
+                                            num_sms, _ptr(dev_status), _stream(stream)))
 
 
-def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, dev_status=None, stream=None):
-    _check("ep_combine", lib().ep_combine(_ptr(y), _ptr(slot), _ptr(topk_w), T, H, k,
+def ep_combine(y, slot, topk_w, T, H, k, out, num_sms=0, dev_status=None, stream=None, *,
+               recv_rows=0):
+    """recv_rows: rows of y (0 = T*k)."""
+    _check("ep_combine", lib().ep_combine(_ptr(y), _ptr(slot), _ptr(topk_w), T, H, k, recv_rows,
                                           _ptr(out), num_sms, _ptr(dev_status),
                                           _stream(stream)))
 
@@ -147,24 +154,33 @@ def ep_dispatch_layout_noalloc(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
 
 def ep_route_layout(logits, bias, T, cfg: RouteCfg, P, R, phys_of, n_rep, max_rep, topk_idx,
                     topk_w, cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
-                    src, workspace, dev_status, stream=None):
+                    src, workspace, dev_status, stream=None, *, row_align=1):
     """ep_route followed by ep_dispatch_layout (one kernel for small batches)."""
     _check("ep_route_layout", lib().ep_route_layout(
-        _ptr(logits), _ptr(bias), T, cfg, P, R, _ptr(phys_of), _ptr(n_rep), max_rep,
+        _ptr(logits), _ptr(bias), T, cfg, P, R, _ptr(phys_of), _ptr(n_rep), max_rep, row_align,
         _ptr(topk_idx), _ptr(topk_w), _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank),
         _ptr(rank_off), _ptr(tok_rank), _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace),
         _ptr(dev_status), _stream(stream)))
 
 
 def ep_dispatch_backward(grad_recv, slot, T, H, k, grad_x, num_sms=0, dev_status=None,
-                         stream=None):
+                         stream=None, *, recv_rows=0):
     _check("ep_dispatch_backward", lib().ep_dispatch_backward(
-        _ptr(grad_recv), _ptr(slot), T, H, k, _ptr(grad_x), num_sms, _ptr(dev_status),
-        _stream(stream)))
+        _ptr(grad_recv), _ptr(slot), T, H, k, recv_rows, _ptr(grad_x), num_sms,
+        _ptr(dev_status), _stream(stream)))
 
 
 def ep_combine_backward(grad_out, y, slot, topk_w, T, H, k, grad_y, grad_w, num_sms=0,
-                        dev_status=None, stream=None):
+                        dev_status=None, stream=None, *, recv_rows=0):
     _check("ep_combine_backward", lib().ep_combine_backward(
-        _ptr(grad_out), _ptr(y), _ptr(slot), _ptr(topk_w), T, H, k, _ptr(grad_y), _ptr(grad_w),
-        num_sms, _ptr(dev_status), _stream(stream)))
+        _ptr(grad_out), _ptr(y), _ptr(slot), _ptr(topk_w), T, H, k, recv_rows, _ptr(grad_y),
+        _ptr(grad_w), num_sms, _ptr(dev_status), _stream(stream)))
+
+
+def ep_silu_mul(gate_up, n_rows, I, expert_off, cnt_expert, P, fp8, act, act_scale, num_sms=0,
+                stream=None):
+    """silu(gate) * up of the rows [expert_off[p], expert_off[p] + cnt_expert[p])
+    (every row when both are None), e4m3 + 1x128 scales when fp8, else bf16."""
+    _check("ep_silu_mul", lib().ep_silu_mul(
+        _ptr(gate_up), n_rows, I, _ptr(expert_off), _ptr(cnt_expert), P, int(bool(fp8)),
+        _ptr(act), _ptr(act_scale), num_sms, _stream(stream)))

@@ -114,7 +114,7 @@ cudaError_t launch_combine_backward(const CombineBackwardArgs &a, cudaStream_t s
     const int blocks = a.T < a.grid ? a.T : a.grid;
     return launch_pdl(combine_backward_kernel, dim3(blocks), dim3(BWD_THREADS), 0, s,
                       static_cast<const uint16_t *>(a.g), static_cast<const uint16_t *>(a.y),
-                      a.slot, a.w, a.T, a.H, a.k, a.T * a.k, static_cast<uint16_t *>(a.grad_y),
+                      a.slot, a.w, a.T, a.H, a.k, a.n_rows, static_cast<uint16_t *>(a.grad_y),
                       a.grad_w);
 }
 

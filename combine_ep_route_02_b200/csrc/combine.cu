@@ -87,7 +87,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s)
     long long blocks = (chunks + COMBINE_THREADS - 1) / COMBINE_THREADS;
     if (blocks > a.grid) blocks = a.grid;
     return launch_pdl(combine_kernel, dim3((int)blocks), dim3(COMBINE_THREADS), 0, s,
-                      static_cast<const uint16_t *>(a.y), a.slot, a.w, a.T, a.H, a.k, a.T * a.k,
+                      static_cast<const uint16_t *>(a.y), a.slot, a.w, a.T, a.H, a.k, a.n_rows,
                       static_cast<uint16_t *>(a.out));
 }
 

@@ -13,84 +13,13 @@
 // amplification costs no extra reads or arithmetic.
 #include "ep_device.cuh"
 #include "ep_internal.h"
+#include "quant.cuh"
 
 namespace ep {
 
 namespace {
 
 constexpr int DISPATCH_THREADS = 256;
-
-// fp32(x / scale), rounded to nearest even, from the block's shared
-// reciprocal rcp = fp32(1 / scale): one product, then Markstein's correction
-// step (P. Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): the residual
-// x - q0 * scale is exact in one FMA and q0 + residual * rcp rounds to the
-// correctly rounded quotient.  Used only for normal scales with a normal
-// reciprocal (see fast_div_ok); the exhaustive dispatch test checks every
-// bf16 (x, amax) pair against the oracle's IEEE division.
-EP_DEV float div_by_scale(float x, float scale, float rcp)
-{
-    const float q0 = __fmul_rn(x, rcp);
-    const float r = __fmaf_rn(-q0, scale, x);
-    // scale > 0, so the quotient carries the sign of x; the correction
-    // would turn x = -0 into +0 (r = +0, then +0 + -0 = +0)
-    return copysignf(__fmaf_rn(r, rcp, q0), x);
-}
-
-// The correction is exact while the residual cannot underflow: for a
-// quotient large enough to reach an e4m3 rounding point (>= 2^-11) the
-// residual is about 2^-23 |x| >= 2^-34 scale, a normal number once
-// scale >= 2^-90; smaller quotients encode to zero either way.  Tinier
-// scales (amax below about 3.6e-25) take the IEEE division.
-EP_DEV bool fast_div_ok(float scale)
-{
-    return scale >= 0x1p-90f && scale <= 0x1p125f;
-}
-
-EP_DEV uint32_t quant4(const float *v, float scale, float rcp, bool fast)
-{
-    // q = e4m3(fp32(x / scale))
-    float q[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = fast ? div_by_scale(v[i], scale, rcp) : __fdiv_rn(v[i], scale);
-    return pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
-}
-
-// Quantise one 16-element chunk (two 16-byte bf16 vectors).  The 8 lanes
-// whose chunks form one 128-element block must call this together (xor
-// shuffles over lane offsets 1, 2, 4); every lane of the warp must call it.
-EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
-{
-    float v[16];
-    v[0] = bf16_lo(lo.x);  v[1] = bf16_hi(lo.x);
-    v[2] = bf16_lo(lo.y);  v[3] = bf16_hi(lo.y);
-    v[4] = bf16_lo(lo.z);  v[5] = bf16_hi(lo.z);
-    v[6] = bf16_lo(lo.w);  v[7] = bf16_hi(lo.w);
-    v[8] = bf16_lo(hi.x);  v[9] = bf16_hi(hi.x);
-    v[10] = bf16_lo(hi.y); v[11] = bf16_hi(hi.y);
-    v[12] = bf16_lo(hi.z); v[13] = bf16_hi(hi.z);
-    v[14] = bf16_lo(hi.w); v[15] = bf16_hi(hi.w);
-
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 4));
-    const float scale = __fdiv_rn(amax, 448.0f);
-    scale_out = scale;
-
-    uint4 q = make_uint4(0, 0, 0, 0);  // amax == 0: scale 0, zero bytes
-    if (amax != 0.0f) {
-        const bool fast = fast_div_ok(scale);
-        const float rcp = fast ? __frcp_rn(scale) : 0.0f;
-        q.x = quant4(v + 0, scale, rcp, fast);
-        q.y = quant4(v + 4, scale, rcp, fast);
-        q.z = quant4(v + 8, scale, rcp, fast);
-        q.w = quant4(v + 12, scale, rcp, fast);
-    }
-    return q;
-}
 
 __global__ void __launch_bounds__(DISPATCH_THREADS)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
@@ -118,7 +47,7 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
             hi = ld_stream(p + 8);
         }
         float scale;
-        const uint4 q = quant_chunk(lo, hi, scale);
+        const uint4 q = quant::quant_chunk(lo, hi, scale);
         if (active) {
             const int32_t *sl = slot + (size_t)t * k;
             for (int j = 0; j < k; ++j) {
@@ -237,7 +166,7 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                 hi = lds128(in + 32u * c + 16u);
             }
             float scale;
-            const uint4 q = quant_chunk(lo, hi, scale);
+            const uint4 q = quant::quant_chunk(lo, hi, scale);
             if (act) {
                 sts128(qo + 16u * c, q);
                 if ((c & 7) == 0)
@@ -320,12 +249,12 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s)
         return launch_pdl(dispatch_fp8_tma_kernel, dim3(blocks), dim3(tma_threads(a.H)),
                           tma_smem_bytes(a.H), s, static_cast<const uint16_t *>(a.x), a.T, a.H,
                           a.k, a.slot, static_cast<uint8_t *>(a.recv_x), a.recv_scale,
-                          a.T * a.k, a.dev_status);
+                          a.n_rows, a.dev_status);
     }
     const long long chunks = (long long)a.T * (a.fp8 ? a.H / 16 : a.H / 8);
     long long blocks = (chunks + DISPATCH_THREADS - 1) / DISPATCH_THREADS;
     if (blocks > a.grid) blocks = a.grid;
-    const int n_rows = a.T * a.k;
+    const int n_rows = a.n_rows;
     if (a.fp8)
         return launch_pdl(dispatch_fp8_kernel, dim3((int)blocks), dim3(DISPATCH_THREADS), 0, s,
                           static_cast<const uint16_t *>(a.x), a.T, a.H, a.k, a.slot,

@@ -106,7 +106,7 @@ ep_status check_route(const float *logits, const float *bias, int T, ep_route_cf
 }
 
 ep_status check_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
-                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep, int row_align,
                        int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
                        int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank, int32_t *slot,
                        int32_t *src, void *workspace, int32_t *dev_status)
@@ -117,7 +117,10 @@ ep_status check_layout(const int32_t *topk_idx, int T, int k, int E, int P, int 
     if (phys_of == nullptr && P != E) return EP_ERR_INVALID;
     if (phys_of != nullptr && (P < E || max_rep < 1)) return EP_ERR_INVALID;
     if (k > MAX_TOPK || P > MAX_PHYS) return EP_ERR_UNSUPPORTED;
+    if (row_align < 1) return EP_ERR_INVALID;
+    if (row_align > MAX_ROW_ALIGN) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || (long long)T * R >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
+    if ((long long)T * k + (long long)P * (row_align - 1) >= (1LL << 31)) return EP_ERR_UNSUPPORTED;
     if (!cnt_expert || !expert_off || !rows_rank || !rank_off || !tok_rank) return EP_ERR_INVALID;
     if (T > 0 && (!topk_idx || !in_rank || !slot || !src || !workspace)) return EP_ERR_INVALID;
     if (!aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(slot, 4) || !aligned(src, 4) ||
@@ -126,8 +129,11 @@ ep_status check_layout(const int32_t *topk_idx, int T, int k, int E, int P, int 
     return EP_OK;
 }
 
+// receive rows of a copy call: recv_rows, or T * k when recv_rows <= 0
+int rows_of(int recv_rows, int T, int k) { return recv_rows > 0 ? recv_rows : T * k; }
+
 LayoutArgs layout_args(const int32_t *topk_idx, int T, int k, int E, int P, int R,
-                       const int32_t *phys_of, const int32_t *n_rep, int max_rep,
+                       const int32_t *phys_of, const int32_t *n_rep, int max_rep, int row_align,
                        int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
                        int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank, int32_t *slot,
                        int32_t *src, void *workspace, int32_t *dev_status)
@@ -140,7 +146,7 @@ LayoutArgs layout_args(const int32_t *topk_idx, int T, int k, int E, int P, int 
                       cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
                       reinterpret_cast<int32_t *>(ws), reinterpret_cast<int32_t *>(ws + o1),
                       reinterpret_cast<int32_t *>(ws + o2), dev_status,
-                      layout_tile_tokens(T, k, P), NT, layout_hist_warps(P)};
+                      layout_tile_tokens(T, k, P), NT, layout_hist_warps(P), row_align};
 }
 
 }  // namespace
@@ -160,40 +166,42 @@ ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg c
 
 ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
                              const int32_t *phys_of, const int32_t *n_rep, int max_rep,
-                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
-                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
-                             int32_t *slot, int32_t *src, void *workspace,
+                             int row_align, int32_t *cnt_expert, int32_t *expert_off,
+                             int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                             uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
                              int32_t *dev_status, ep_stream_t stream)
 {
-    const ep_status st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
+    const ep_status st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align,
                                       cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
                                       in_rank, slot, src, workspace, dev_status);
     if (st != EP_OK) return st;
-    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
-                                     expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
-                                     src, workspace, dev_status);
+    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align,
+                                     cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
+                                     in_rank, slot, src, workspace, dev_status);
     return from_cuda(launch_layout(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_route_cfg cfg,
                           int P, int R, const int32_t *phys_of, const int32_t *n_rep,
-                          int max_rep, int32_t *topk_idx, float *topk_w, int32_t *cnt_expert,
-                          int32_t *expert_off, int32_t *rows_rank, int32_t *rank_off,
+                          int max_rep, int row_align, int32_t *topk_idx, float *topk_w,
+                          int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
+                          int32_t *rank_off,
                           int32_t *tok_rank, uint8_t *in_rank, int32_t *slot, int32_t *src,
                           void *workspace, int32_t *dev_status, ep_stream_t stream)
 {
     ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
     if (st != EP_OK) return st;
     const int E = cfg.num_experts, k = cfg.topk;
-    st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert, expert_off,
-                      rows_rank, rank_off, tok_rank, in_rank, slot, src, workspace, dev_status);
+    st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align, cnt_expert,
+                      expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src, workspace,
+                      dev_status);
     if (st != EP_OK) return st;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const RouteArgs r{logits, bias, T, E, cfg.n_group, cfg.topk_group, k, cfg.routed_scale,
                       cfg.renorm != 0, topk_idx, topk_w};
-    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
-                                     expert_off, rows_rank, rank_off, tok_rank, in_rank, slot,
-                                     src, workspace, dev_status);
+    const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align,
+                                     cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
+                                     in_rank, slot, src, workspace, dev_status);
     if (small_route_layout_ok(T, k, P)) {
         int *done = reinterpret_cast<int *>(static_cast<char *>(workspace) +
                                             layout_workspace_core(T, k, P, R));
@@ -204,9 +212,9 @@ ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_rout
     return from_cuda(launch_layout(a, s));
 }
 
-ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
-                      void *recv_x, float *recv_scale, int num_sms, int32_t *dev_status,
-                      ep_stream_t stream)
+ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
+                      const int32_t *slot, int fp8, void *recv_x, float *recv_scale, int num_sms,
+                      int32_t *dev_status, ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1) return EP_ERR_INVALID;
     if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_INVALID;
@@ -217,13 +225,15 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *sl
         !aligned(dev_status, 4))
         return EP_ERR_INVALID;
     DispatchArgs a{x_bf16, T, H, k, slot, fp8 != 0, recv_x, recv_scale,
-                   streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0)), 0, dev_status};
+                   streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0)), 0, dev_status,
+                   rows_of(recv_rows, T, k)};
     if (T > 0 && dispatch_tma_ok(a)) a.tma_grid = streaming_grid(num_sms, tma_blocks_per_sm(H));
     return from_cuda(launch_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T, int H,
-                     int k, void *out_bf16, int num_sms, int32_t *dev_status, ep_stream_t stream)
+                     int k, int recv_rows, void *out_bf16, int num_sms, int32_t *dev_status,
+                     ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
@@ -233,13 +243,13 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
         !aligned(dev_status, 4))
         return EP_ERR_INVALID;
     CombineArgs a{y_bf16, slot, topk_w, T, H, k, out_bf16,
-                  streaming_grid(num_sms, cached_blocks_per_sm(2))};
+                  streaming_grid(num_sms, cached_blocks_per_sm(2)), rows_of(recv_rows, T, k)};
     return from_cuda(launch_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, int T, int H,
-                               int k, void *grad_x_bf16, int num_sms, int32_t *dev_status,
-                               ep_stream_t stream)
+                               int k, int recv_rows, void *grad_x_bf16, int num_sms,
+                               int32_t *dev_status, ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
@@ -249,13 +259,13 @@ ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, 
         !aligned(dev_status, 4))
         return EP_ERR_INVALID;
     CombineArgs a{grad_recv_bf16, slot, nullptr, T, H, k, grad_x_bf16,
-                  streaming_grid(num_sms, cached_blocks_per_sm(2))};
+                  streaming_grid(num_sms, cached_blocks_per_sm(2)), rows_of(recv_rows, T, k)};
     return from_cuda(launch_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, const int32_t *slot,
-                              const float *topk_w, int T, int H, int k, void *grad_y_bf16,
-                              float *grad_w, int num_sms, int32_t *dev_status,
+                              const float *topk_w, int T, int H, int k, int recv_rows,
+                              void *grad_y_bf16, float *grad_w, int num_sms, int32_t *dev_status,
                               ep_stream_t stream)
 {
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
@@ -275,8 +285,34 @@ ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, con
         if (dev < 64) occ[dev] = per_sm;
     }
     CombineBackwardArgs a{grad_out_bf16, y_bf16, slot, topk_w, T, H, k, grad_y_bf16, grad_w,
-                          streaming_grid(num_sms, per_sm)};
+                          streaming_grid(num_sms, per_sm), rows_of(recv_rows, T, k)};
     return from_cuda(launch_combine_backward(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_silu_mul(const void *gate_up_bf16, int n_rows, int I, const int32_t *expert_off,
+                      const int32_t *cnt_expert, int P, int fp8, void *act, float *act_scale,
+                      int num_sms, ep_stream_t stream)
+{
+    if (n_rows < 0 || I < 1 || I % 128 != 0) return EP_ERR_INVALID;
+    if ((expert_off == nullptr) != (cnt_expert == nullptr)) return EP_ERR_INVALID;
+    if (expert_off != nullptr && P < 1) return EP_ERR_INVALID;
+    if (P > MAX_PHYS) return EP_ERR_UNSUPPORTED;
+    if ((long long)n_rows * 2 * I >= (1LL << 40)) return EP_ERR_UNSUPPORTED;
+    if (n_rows > 0 && (!gate_up_bf16 || !act || (fp8 && !act_scale))) return EP_ERR_INVALID;
+    if (!aligned(gate_up_bf16, 16) || !aligned(act, 16) || !aligned(act_scale, 4) ||
+        !aligned(expert_off, 4) || !aligned(cnt_expert, 4))
+        return EP_ERR_INVALID;
+    static volatile int occ[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int per_sm = dev < 64 ? occ[dev] : 0;
+    if (per_sm <= 0) {
+        per_sm = activation_blocks_per_sm();
+        if (dev < 64) occ[dev] = per_sm;
+    }
+    ActivationArgs a{gate_up_bf16, n_rows, I, expert_off, cnt_expert, expert_off ? P : 0,
+                     fp8 != 0, act, act_scale, streaming_grid(num_sms, per_sm)};
+    return from_cuda(launch_activation(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -20,6 +20,7 @@ constexpr int MAX_EXPERTS = 1024;   // logical experts (routing)
 constexpr int MAX_PHYS = 4096;      // physical experts (layout)
 constexpr int MAX_TOPK = 32;
 constexpr int MAX_GROUPS = 32;
+constexpr int MAX_ROW_ALIGN = 1024;  // GEMM row tile of the padded layout
 
 struct RouteArgs {
     const float *logits;
@@ -47,6 +48,7 @@ struct LayoutArgs {
     int tile_tokens;    // TT
     int n_tiles;        // NT
     int hist_warps;     // slot-kernel warps that order pairs
+    int row_align;      // each expert's first receive row is a multiple of this
 };
 
 struct DispatchArgs {
@@ -59,6 +61,7 @@ struct DispatchArgs {
     int grid;          // register-path grid
     int tma_grid;      // > 0: use the TMA pipeline with this many CTAs
     int32_t *dev_status;
+    int n_rows;        // receive rows; slots outside [0, n_rows) are skipped
 };
 
 struct CombineArgs {
@@ -68,6 +71,7 @@ struct CombineArgs {
     int T, H, k;
     void *out;
     int grid;
+    int n_rows;        // rows of y; slots outside [0, n_rows) are skipped
 };
 
 // Warps of the slot kernel that each order one contiguous share of a tile's
@@ -105,8 +109,23 @@ struct CombineBackwardArgs {
     const int32_t *slot;
     const float *w;
     int T, H, k;
-    void *grad_y;      // bf16 [T*k, H]
+    void *grad_y;      // bf16 [n_rows, H]
     float *grad_w;     // [T, k]
+    int grid;
+    int n_rows;        // rows of y and grad_y
+};
+
+// Expert activation: h = silu(gate) * up over the rows the per-expert counts
+// select, quantised to e4m3 with 1x128 scales (or stored as bf16).
+struct ActivationArgs {
+    const void *gate_up;       // bf16 [n_rows, 2I]
+    int n_rows, I;
+    const int32_t *expert_off; // [P+1] or null (every row)
+    const int32_t *cnt_expert; // [P]
+    int P;
+    int fp8;
+    void *act;                 // e4m3 [n_rows, I] or bf16 [n_rows, I]
+    float *act_scale;          // [n_rows, I/128] when fp8
     int grid;
 };
 
@@ -159,6 +178,8 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
 cudaError_t launch_combine_backward(const CombineBackwardArgs &a, cudaStream_t s);
 int combine_backward_blocks_per_sm();
+cudaError_t launch_activation(const ActivationArgs &a, cudaStream_t s);
+int activation_blocks_per_sm();
 
 // resident blocks per SM for each streaming kernel at its block size
 int dispatch_blocks_per_sm(int fp8);

@@ -244,6 +244,13 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
             if (threadIdx.x == 0) *a.dev_status = st;
         }
     }
+    if (a.row_align > 1) {
+        // GEMM layout: every expert's rows start on a multiple of the row
+        // tile (same thread-to-expert mapping as the loops above)
+        const int A = a.row_align;
+        for (int p = threadIdx.x; p < a.P; p += blockDim.x) eoff[p] = (eoff[p] + A - 1) / A * A;
+        __syncthreads();
+    }
     const int total = block_exclusive_scan<NTHREADS>(eoff, a.P, warp_tot);
     if (threadIdx.x == 0) eoff[a.P] = total;
     __syncthreads();
@@ -256,6 +263,15 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
             a.rows_rank[r] = eoff[(r + 1) * epr] - eoff[r * epr];
         }
         if (threadIdx.x == 0) a.rank_off[a.R] = total;
+        if (a.row_align > 1) {
+            // padding rows after each expert's pairs: src = -1 (a warp per
+            // expert; cnt_expert was written by this block above, or by the
+            // scan kernel)
+            for (int p = warp; p < a.P; p += NWARPS) {
+                const int first = eoff[p] + a.cnt_expert[p];
+                for (int r = first + lane; r < eoff[p + 1]; r += 32) a.src[r] = -1;
+            }
+        }
     }
 
     // warps w < HW each own a contiguous share of the tile's pairs, in (t, j)

@@ -56,7 +56,7 @@ extern "C" ep_status ep_dispatch_layout_noalloc(
     if (scratch_address(&scratch) != cudaSuccess) return EP_ERR_CUDA;
     // the layout kernels overwrite every scratch word they read, so the
     // previous call's contents need no clearing
-    return ep_dispatch_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, cnt_expert,
+    return ep_dispatch_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, 1, cnt_expert,
                               expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src,
                               scratch, dev_status, stream);
 }

@@ -20,17 +20,19 @@ from . import _binding as B
 class EpPath:
     """Buffers and calls for one (T, H, routing, ranks) shape.
 
-    The receive buffers have T*k rows: rank r's rows are
-    ``recv_x[rank_off[r]:rank_off[r+1]]`` and expert p's rows are
-    ``recv_x[expert_off[p]:expert_off[p+1]]``.
+    The receive buffers have ``n_recv`` rows: T*k, plus P*(row_align-1) when
+    each expert's rows start on a multiple of ``row_align`` (the GEMM layout).
+    Rank r's rows are ``recv_x[rank_off[r]:rank_off[r+1]]`` and expert p's
+    pairs are ``recv_x[expert_off[p]:expert_off[p] + cnt_expert[p]]``.
     """
 
     def __init__(self, T: int, H: int, num_experts: int, n_group: int, topk_group: int,
                  topk: int, routed_scale: float, renorm: bool, R: int, fp8: bool,
                  phys_of: Optional[torch.Tensor] = None, n_rep: Optional[torch.Tensor] = None,
-                 device="cuda", num_sms: int = 0):
+                 device="cuda", num_sms: int = 0, row_align: int = 1):
         dev = torch.device(device)
         self.T, self.H, self.k, self.E, self.R = T, H, topk, num_experts, R
+        self.row_align = int(row_align)
         self.fp8 = bool(fp8)
         self.num_sms = num_sms          # SMs for dispatch and combine (0 = all)
         self.dispatch_sms = num_sms
@@ -47,6 +49,7 @@ class EpPath:
             self.max_rep = 0
             self.P = num_experts
         P, k = self.P, topk
+        self.n_recv = T * k + P * (self.row_align - 1)
         i32 = dict(device=dev, dtype=torch.int32)
         self.topk_idx = torch.empty((T, k), **i32)
         self.topk_w = torch.empty((T, k), device=dev, dtype=torch.float32)
@@ -57,16 +60,17 @@ class EpPath:
         self.tok_rank = torch.empty(R, **i32)
         self.in_rank = torch.empty((T, R), device=dev, dtype=torch.uint8)
         self.slot = torch.empty((T, k), **i32)
-        self.src = torch.empty(T * k, **i32)
+        self.src = torch.empty(self.n_recv, **i32)
         self.dev_status = torch.zeros(1, **i32)    # layout (cleared by each layout call)
         self.copy_status = torch.zeros(1, **i32)   # dispatch / combine (sticky)
         ws = B.ep_workspace_size(T, k, P, R)
         self.workspace = torch.empty(max(ws, 256), device=dev, dtype=torch.uint8)
+        n = self.n_recv
         if self.fp8:
-            self.recv_x = torch.empty((T * k, H), device=dev, dtype=torch.float8_e4m3fn)
-            self.recv_scale = torch.empty((T * k, H // 128), device=dev, dtype=torch.float32)
+            self.recv_x = torch.empty((n, H), device=dev, dtype=torch.float8_e4m3fn)
+            self.recv_scale = torch.empty((n, H // 128), device=dev, dtype=torch.float32)
         else:
-            self.recv_x = torch.empty((T * k, H), device=dev, dtype=torch.bfloat16)
+            self.recv_x = torch.empty((n, H), device=dev, dtype=torch.bfloat16)
             self.recv_scale = None
         self.out = torch.empty((T, H), device=dev, dtype=torch.bfloat16)
 
@@ -79,7 +83,7 @@ class EpPath:
                              self.phys_of, self.n_rep, self.max_rep, self.cnt_expert,
                              self.expert_off, self.rows_rank, self.rank_off, self.tok_rank,
                              self.in_rank, self.slot, self.src, self.workspace,
-                             self.dev_status, stream)
+                             self.dev_status, stream, row_align=self.row_align)
 
     def route_layout(self, logits: torch.Tensor, bias: Optional[torch.Tensor], stream=None):
         """route then layout in one call (one kernel for small batches)"""
@@ -87,17 +91,29 @@ class EpPath:
                           self.n_rep, self.max_rep, self.topk_idx, self.topk_w,
                           self.cnt_expert, self.expert_off, self.rows_rank, self.rank_off,
                           self.tok_rank, self.in_rank, self.slot, self.src, self.workspace,
-                          self.dev_status, stream)
+                          self.dev_status, stream, row_align=self.row_align)
 
     def dispatch(self, x: torch.Tensor, stream=None):
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
-                      self.recv_scale, self.dispatch_sms, self.copy_status, stream)
+                      self.recv_scale, self.dispatch_sms, self.copy_status, stream,
+                      recv_rows=self.n_recv)
 
     def combine(self, y: torch.Tensor, stream=None, out: Optional[torch.Tensor] = None):
+        """y: expert outputs, ``n_recv`` rows in receive-row order."""
         out = self.out if out is None else out
         B.ep_combine(y, self.slot, self.topk_w, self.T, self.H, self.k, out,
-                     self.combine_sms, self.copy_status, stream)
+                     self.combine_sms, self.copy_status, stream, recv_rows=self.n_recv)
         return out
+
+    def activation(self, gate_up: torch.Tensor, act: torch.Tensor,
+                   act_scale: Optional[torch.Tensor], stream=None):
+        """silu(gate) * up of the filled receive rows (the counts of the last
+        layout, read on the device); ``gate_up`` bf16 [n_recv, 2I], ``act``
+        e4m3 [n_recv, I] with ``act_scale`` fp32 [n_recv, I/128], or bf16
+        [n_recv, I] with ``act_scale`` None."""
+        I = gate_up.shape[1] // 2
+        B.ep_silu_mul(gate_up, self.n_recv, I, self.expert_off, self.cnt_expert, self.P,
+                      act_scale is not None, act, act_scale, self.num_sms, stream)
 
     def step(self, x, logits, bias, y, stream=None, out=None):
         """route, layout, dispatch, then combine of the expert outputs y."""

@@ -171,6 +171,7 @@ class WorkloadConfig:
     n_hot: int = 0
     zipf_s: float = 1.2
     zipf_beta: float = 0.05
+    inter: int = 2048        # expert intermediate width I (gate and up halves)
 
     @property
     def n_phys(self) -> int:
@@ -183,10 +184,10 @@ class WorkloadConfig:
 CONFIGS = {
     "tiny": WorkloadConfig("tiny", T=128, H=256, E=16, R=4, n_group=1,
                            topk_group=1, topk=2, fp8=False, routed_scale=1.0,
-                           renorm=True, bias="zero"),
+                           renorm=True, bias="zero", inter=128),
     "ds16b": WorkloadConfig("ds16b", T=4096, H=2048, E=64, R=8, n_group=1,
                             topk_group=1, topk=6, fp8=True, routed_scale=1.0,
-                            renorm=True, bias="uniform"),
+                            renorm=True, bias="uniform", inter=1408),
     "v3": WorkloadConfig("v3", T=8192, H=7168, E=256, R=8, n_group=8,
                          topk_group=4, topk=8, fp8=True, routed_scale=2.5,
                          renorm=True, bias="uniform"),

@@ -11,6 +11,8 @@
  *                                      rows (BF16 copies, or e4m3 + 1x128
  *                                      scales)
  *   ep_combine          expert rows -> top-k weighted sum per token (BF16)
+ *   ep_silu_mul         expert intermediate rows -> silu(gate) * up, e4m3 +
+ *                                      1x128 scales for the second expert GEMM
  *
  * Sources (page title, then section):
  *  - Perplexity, "Lower latency and higher throughput with multi-node
@@ -131,27 +133,38 @@ ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg c
  *   phys_of    int32 [E, max_rep] or NULL: physical ids of each expert's
  *              replicas; token t uses replica phys_of[e][t % n_rep[e]]
  *   n_rep      int32 [E] or NULL (together with phys_of)
- *   outputs    cnt_expert [P]     rows per physical expert
- *              expert_off [P+1]   exclusive prefix sum of cnt_expert
- *              rows_rank  [R]     rows per rank (sum of its experts' counts)
+ *   row_align  A, 1..1024: the GEMM layout of the DeepEP V2 summary (its
+ *              feature list names a new GEMM layout).  Each expert's first
+ *              receive row is a multiple of A (the row tile of a grouped GEMM
+ *              reading the receive buffer); A = 1 packs the rows.
+ *   outputs    cnt_expert [P]     rows per physical expert (pairs, unpadded)
+ *              expert_off [P+1]   first row of each expert:
+ *                                 expert_off[p+1] = expert_off[p] +
+ *                                 round_up(cnt_expert[p], A)
+ *              rows_rank  [R]     rows per rank (its experts' padded rows)
  *              rank_off   [R+1]   exclusive prefix sum of rows_rank
  *              tok_rank   [R]     tokens with at least one expert on the rank
  *              in_rank    uint8 [T, R]  1 if token t sends to rank r
  *              slot       [T, k]  receive row of pair (t, j); -1 if invalid
- *              src        [T*k]   inverse of slot: src[slot[t,j]] = t*k + j
+ *              src        [T*k + P*(A-1)] for rows [0, expert_off[P]):
+ *                                 src[slot[t,j]] = t*k + j, and -1 for the
+ *                                 padding rows that follow each expert's pairs
  *   workspace  ep_workspace_size(T, k, P, R) bytes, 256-byte aligned
  *   dev_status int32 [1] or NULL; zeroed by this call, then EP_DEV_* bits
  *
  * Receive rows are ordered by physical expert, and within an expert by
- * (t, j); there is no padding, so valid pairs fill rows [0, expert_off[P]).
- * Rank r's rows are [rank_off[r], rank_off[r+1]).  The result does not
- * depend on scheduling (no global atomics decide an order).
+ * (t, j).  Expert p's pairs fill rows [expert_off[p], expert_off[p] +
+ * cnt_expert[p]); with A = 1 there is no padding and valid pairs fill rows
+ * [0, expert_off[P]).  A receive buffer of T*k + P*(A-1) rows holds any
+ * routing.  Rank r's rows are [rank_off[r], rank_off[r+1]).  The result
+ * does not depend on scheduling (no global atomics decide an order).
+ * T*k + P*(A-1) >= 2^31 returns EP_ERR_UNSUPPORTED.
  */
 ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P, int R,
                              const int32_t *phys_of, const int32_t *n_rep, int max_rep,
-                             int32_t *cnt_expert, int32_t *expert_off, int32_t *rows_rank,
-                             int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank,
-                             int32_t *slot, int32_t *src, void *workspace,
+                             int row_align, int32_t *cnt_expert, int32_t *expert_off,
+                             int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                             uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
                              int32_t *dev_status, ep_stream_t stream);
 
 /*
@@ -168,7 +181,7 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
  */
 ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_route_cfg cfg,
                           int P, int R, const int32_t *phys_of, const int32_t *n_rep,
-                          int max_rep, int32_t *topk_idx, float *topk_w, int32_t *cnt_expert,
+                          int max_rep, int row_align, int32_t *topk_idx, float *topk_w, int32_t *cnt_expert,
                           int32_t *expert_off, int32_t *rows_rank, int32_t *rank_off,
                           int32_t *tok_rank, uint8_t *in_rank, int32_t *slot, int32_t *src,
                           void *workspace, int32_t *dev_status, ep_stream_t stream);
@@ -177,9 +190,11 @@ ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_rout
  * Dispatch (permute, optionally with fused 1x128 FP8 quantisation).
  *
  *   x_bf16      bf16 [T, H], 16-byte aligned; H % 8 == 0 (H % 128 == 0 for fp8)
+ *   recv_rows   N, rows of the receive buffer; N <= 0 means T*k (the packed
+ *               layout); a padded layout needs up to T*k + P*(row_align-1)
  *   slot        int32 [T, k] from ep_dispatch_layout (or a cached copy)
- *   fp8 == 0:   recv_x is bf16 [T*k, H]; row slot[t,j] = x[t] bit for bit
- *   fp8 != 0:   recv_x is e4m3fn [T*k, H] and recv_scale fp32 [T*k, H/128];
+ *   fp8 == 0:   recv_x is bf16 [N, H]; row slot[t,j] = x[t] bit for bit
+ *   fp8 != 0:   recv_x is e4m3fn [N, H] and recv_scale fp32 [N, H/128];
  *               per 128-element block b of x[t]: amax = max|x|, scale =
  *               fp32(amax / 448), q = e4m3_rn_satfinite(fp32(x / scale));
  *               a block with amax == 0 gets scale 0 and zero bytes
@@ -187,30 +202,31 @@ ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_rout
  *   dev_status  int32 [1] or NULL: EP_DEV_TIMEOUT is ORed in if a bounded
  *               wait on a TMA copy gives up (the word is not cleared here)
  *
- * Slots outside [0, T*k) are skipped (rows they would fill are left as they
- * were).  recv_x must be 16-byte aligned, recv_scale 4-byte aligned.  With
+ * Slots outside [0, N) are skipped, and rows no slot names (padding) are
+ * left as they were.  recv_x must be 16-byte aligned, recv_scale 4-byte aligned.  With
  * fp8, H % 512 == 0 and a 16-byte aligned recv_scale, rows move through
  * shared memory by TMA bulk copies; otherwise by 16-byte thread stores.
  */
-ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, const int32_t *slot, int fp8,
-                      void *recv_x, float *recv_scale, int num_sms, int32_t *dev_status,
-                      ep_stream_t stream);
+ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
+                      const int32_t *slot, int fp8, void *recv_x, float *recv_scale, int num_sms,
+                      int32_t *dev_status, ep_stream_t stream);
 
 /*
  * Combine: weighted gather-reduce back to token order.
  *
- *   y_bf16    bf16 [T*k, H] expert outputs in receive-row order
+ *   y_bf16    bf16 [N, H] expert outputs in receive-row order
  *   slot      int32 [T, k], topk_w fp32 [T, k]
+ *   recv_rows N, rows of y (N <= 0 means T*k), as for ep_dispatch
  *   out_bf16  bf16 [T, H] (out)
  *
  * out[t] = bf16_rne( acc ), acc = fp32 sum over j = 0..k-1 in order of
  * fp32(w[t,j] * y[slot[t,j]]), each step rounded to nearest even.  Slots
- * outside [0, T*k) contribute nothing.  y and out 16-byte aligned, H % 8 == 0.
+ * outside [0, N) contribute nothing; padding rows are never read.  y and out 16-byte aligned, H % 8 == 0.
  * dev_status as for ep_dispatch (NULL allowed).
  */
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T,
-                     int H, int k, void *out_bf16, int num_sms, int32_t *dev_status,
-                     ep_stream_t stream);
+                     int H, int k, int recv_rows, void *out_bf16, int num_sms,
+                     int32_t *dev_status, ep_stream_t stream);
 
 /*
  * Allocation-free variant of ep_dispatch_layout.  It has no counterpart in
@@ -220,8 +236,8 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
  * caching allocator), or a latency-bound decode step that cannot afford the
  * device-wide synchronisation cudaMalloc may cause.
  *
- * Arguments and results are those of ep_dispatch_layout without
- * `workspace`: the scratch lives in a fixed __device__ array of
+ * Arguments and results are those of ep_dispatch_layout with row_align = 1
+ * and without `workspace`: the scratch lives in a fixed __device__ array of
  * EP_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
  * the library keeps until the process exits.  Sizes whose
  * ep_workspace_size(T, k, P, R) exceeds that limit return
@@ -248,28 +264,61 @@ ep_status ep_dispatch_layout_noalloc(const int32_t *topk_idx, int T, int k, int 
  * combine.  grad_x[t] = bf16( sum_j grad_recv[slot[t,j]] ), fp32 in j order:
  * ep_combine with unit weights.  With an FP8 forward dispatch the
  * quantisation is treated as the identity; gradients travel in BF16.
- *   grad_recv_bf16  bf16 [T*k, H] gradients of the receive rows
+ *   grad_recv_bf16  bf16 [N, H] gradients of the receive rows
+ *   recv_rows       N (N <= 0 means T*k), as for ep_combine
  *   grad_x_bf16     bf16 [T, H] (out)
  * Alignment, slot handling and dev_status as for ep_combine.
  */
 ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, int T, int H,
-                               int k, void *grad_x_bf16, int num_sms, int32_t *dev_status,
-                               ep_stream_t stream);
+                               int k, int recv_rows, void *grad_x_bf16, int num_sms,
+                               int32_t *dev_status, ep_stream_t stream);
 
 /*
  * Backward of combine (training): combine's backward is a dispatch (same
  * section).  For out[t] = sum_j w[t,j] y[slot[t,j]]:
- *   grad_y[slot[t,j]] = bf16( fp32(w[t,j] * grad_out[t]) )   bf16 [T*k, H]
+ *   grad_y[slot[t,j]] = bf16( fp32(w[t,j] * grad_out[t]) )   bf16 [N, H]
  *   grad_w[t,j]       = sum_h grad_out[t,h] * y[slot[t,j],h]  fp32 [T, k]
+ * with y bf16 [N, H] and N = recv_rows (N <= 0 means T*k).
  * The dot products are accumulated in fp32 in an unspecified order (within
  * about 1e-5 of the sum of |terms| of the exact value).  Rows of invalid
  * slots are not written and their grad_w is 0.  16-byte alignment for the
  * bf16 arrays; dev_status as for ep_combine.
  */
 ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, const int32_t *slot,
-                              const float *topk_w, int T, int H, int k, void *grad_y_bf16,
-                              float *grad_w, int num_sms, int32_t *dev_status,
+                              const float *topk_w, int T, int H, int k, int recv_rows,
+                              void *grad_y_bf16, float *grad_w, int num_sms, int32_t *dev_status,
                               ep_stream_t stream);
+
+/*
+ * Expert activation between the two grouped GEMMs of a gated-SiLU expert,
+ * with the 1x128 FP8 quantisation the second GEMM reads (Perplexity blog,
+ * section "Quantization": the SiLU kernel works under CUDA graphs, with
+ * block quantisation and a routed token count known only on the device, so
+ * a fixed set of persistent blocks reads the per-expert counts and shares
+ * out the filled rows).
+ *
+ *   gate_up_bf16  bf16 [n_rows, 2I]: row r = [gate (I) | up (I)], the first
+ *                 GEMM's output in receive-row order; 16-byte aligned
+ *   I             intermediate width, I % 128 == 0
+ *   expert_off    int32 [P+1] and cnt_expert int32 [P] from
+ *                 ep_dispatch_layout (device memory, read by the kernel):
+ *                 rows [expert_off[p], expert_off[p] + cnt_expert[p]) are
+ *                 processed, padding and unused rows are not touched.  Both
+ *                 NULL: every one of the n_rows rows is processed.
+ *   fp8 != 0:     act is e4m3fn [n_rows, I] and act_scale fp32 [n_rows, I/128]
+ *   fp8 == 0:     act is bf16 [n_rows, I] holding h itself (act_scale unused)
+ *
+ * Per element: s = bf16(silu(g)) with silu(g) = g / (1 + e^-g) correctly
+ * rounded (silu(-inf) = -0); h = bf16(fp32(s * u)), each rounding to nearest
+ * even.  Per 128-element block of h: amax = max |h| (NaN ignored), scale =
+ * fp32(amax / 448), q = e4m3_rn_satfinite(fp32(h / scale)); amax == 0 gives
+ * scale 0 and zero bytes.  Rows from offsets outside [0, n_rows) are skipped.
+ * The launch size depends on num_sms only, never on the counts, so the call
+ * can be captured in a CUDA graph with the counts changing between replays.
+ */
+ep_status ep_silu_mul(const void *gate_up_bf16, int n_rows, int I, const int32_t *expert_off,
+                      const int32_t *cnt_expert, int P, int fp8, void *act, float *act_scale,
+                      int num_sms, ep_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char *ep_status_string(ep_status status);

@@ -25,11 +25,11 @@ def bf16_from_bits(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
 
 
-def make_path(cfg, wl: Workload, num_sms: int = 0):
+def make_path(cfg, wl: Workload, num_sms: int = 0, row_align: int = 1):
     from combine_ep_route_02_b200 import EpPath
     return EpPath(cfg.T, cfg.H, cfg.E, cfg.n_group, cfg.topk_group, cfg.topk,
                   cfg.routed_scale, cfg.renorm, cfg.R, cfg.fp8,
-                  phys_of=wl.phys_of, n_rep=wl.n_rep, num_sms=num_sms)
+                  phys_of=wl.phys_of, n_rep=wl.n_rep, num_sms=num_sms, row_align=row_align)
 
 
 def oracle_route(cfg, wl):
@@ -37,10 +37,10 @@ def oracle_route(cfg, wl):
                         cfg.routed_scale, cfg.renorm)
 
 
-def oracle_layout(cfg, wl, topk_idx):
+def oracle_layout(cfg, wl, topk_idx, row_align: int = 1):
     po = None if wl.phys_of is None else wl.phys_of.numpy()
     nr = None if wl.n_rep is None else wl.n_rep.numpy()
-    return oracle.layout(topk_idx, cfg.E, cfg.n_phys, cfg.R, po, nr)
+    return oracle.layout(topk_idx, cfg.E, cfg.n_phys, cfg.R, po, nr, row_align=row_align)
 
 
 LAYOUT_FIELDS = ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank",

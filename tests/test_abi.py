@@ -78,14 +78,14 @@ def test_route_rejects_unsupported(lib, kw):
     assert st in (B.EP_ERR_UNSUPPORTED, B.EP_ERR_INVALID) and st != B.EP_OK
 
 
-def layout(lib, T=4, k=2, E=16, P=16, R=4, phys=None, nrep=None, ws=FAKE, max_rep=0):
-    return lib.ep_dispatch_layout(FAKE, T, k, E, P, R, phys, nrep, max_rep, FAKE, FAKE, FAKE,
-                                  FAKE, FAKE, FAKE, FAKE, FAKE, ws, None, None)
+def layout(lib, T=4, k=2, E=16, P=16, R=4, phys=None, nrep=None, ws=FAKE, max_rep=0, align=1):
+    return lib.ep_dispatch_layout(FAKE, T, k, E, P, R, phys, nrep, max_rep, align, FAKE, FAKE,
+                                  FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None, None)
 
 
 @pytest.mark.parametrize("kw", [
     dict(P=16, R=3), dict(P=20), dict(phys=FAKE), dict(phys=FAKE, nrep=FAKE, max_rep=0),
-    dict(ws=FAKE + 16), dict(T=-2), dict(k=0),
+    dict(ws=FAKE + 16), dict(T=-2), dict(k=0), dict(align=0), dict(align=-4),
 ])
 def test_layout_rejects_invalid(lib, kw):
     assert layout(lib, **kw) == B.EP_ERR_INVALID
@@ -95,26 +95,51 @@ def test_layout_rejects_too_many_experts(lib):
     assert layout(lib, E=5000, P=5000, R=8) == B.EP_ERR_UNSUPPORTED
 
 
+def test_layout_rejects_unsupported_alignment(lib):
+    assert layout(lib, align=2048) == B.EP_ERR_UNSUPPORTED
+    # T*k + P*(A-1) rows must stay below 2^31
+    T = (1 << 31) // 16 - 100                    # T*k fits, the padding does not
+    assert layout(lib, T=T, k=16, E=4096, P=4096, R=8, align=1024) == B.EP_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("args", [
-    (FAKE, 4, 100, 2, FAKE, 1, FAKE, FAKE),    # fp8 needs H % 128 == 0
-    (FAKE, 4, 100, 2, FAKE, 0, FAKE, None),    # bf16 needs H % 8 == 0
-    (MIS, 4, 256, 2, FAKE, 1, FAKE, FAKE),     # x not 16-byte aligned
-    (FAKE, 4, 256, 2, FAKE, 1, MIS, FAKE),     # recv_x not 16-byte aligned
-    (FAKE, 4, 256, 2, FAKE, 1, FAKE, None),    # fp8 without a scale buffer
-    (FAKE, 4, 256, 0, FAKE, 1, FAKE, FAKE),
+    (FAKE, 4, 100, 2, 0, FAKE, 1, FAKE, FAKE),    # fp8 needs H % 128 == 0
+    (FAKE, 4, 100, 2, 0, FAKE, 0, FAKE, None),    # bf16 needs H % 8 == 0
+    (MIS, 4, 256, 2, 0, FAKE, 1, FAKE, FAKE),     # x not 16-byte aligned
+    (FAKE, 4, 256, 2, 0, FAKE, 1, MIS, FAKE),     # recv_x not 16-byte aligned
+    (FAKE, 4, 256, 2, 0, FAKE, 1, FAKE, None),    # fp8 without a scale buffer
+    (FAKE, 4, 256, 0, 0, FAKE, 1, FAKE, FAKE),
 ])
 def test_dispatch_rejects_invalid(lib, args):
     assert lib.ep_dispatch(*args, 0, None, None) == B.EP_ERR_INVALID
 
 
 @pytest.mark.parametrize("args", [
-    (FAKE, FAKE, FAKE, 4, 100, 2, FAKE),
-    (MIS, FAKE, FAKE, 4, 256, 2, FAKE),
-    (FAKE, FAKE, FAKE, 4, 256, 2, MIS),
-    (FAKE, FAKE, FAKE, -1, 256, 2, FAKE),
+    (FAKE, FAKE, FAKE, 4, 100, 2, 0, FAKE),
+    (MIS, FAKE, FAKE, 4, 256, 2, 0, FAKE),
+    (FAKE, FAKE, FAKE, 4, 256, 2, 0, MIS),
+    (FAKE, FAKE, FAKE, -1, 256, 2, 0, FAKE),
 ])
 def test_combine_rejects_invalid(lib, args):
     assert lib.ep_combine(*args, 0, None, None) == B.EP_ERR_INVALID
+
+
+@pytest.mark.parametrize("args", [
+    (FAKE, 4, 100, None, None, 0, 1, FAKE, FAKE),     # I % 128 != 0
+    (FAKE, 4, 256, FAKE, None, 16, 1, FAKE, FAKE),    # offsets without counts
+    (FAKE, 4, 256, FAKE, FAKE, 0, 1, FAKE, FAKE),     # counts for no experts
+    (MIS, 4, 256, None, None, 0, 1, FAKE, FAKE),      # gate_up misaligned
+    (FAKE, 4, 256, None, None, 0, 1, MIS, FAKE),      # act misaligned
+    (FAKE, 4, 256, None, None, 0, 1, FAKE, None),     # fp8 without scales
+    (FAKE, -1, 256, None, None, 0, 1, FAKE, FAKE),
+])
+def test_silu_mul_rejects_invalid(lib, args):
+    assert lib.ep_silu_mul(*args, 0, None) == B.EP_ERR_INVALID
+
+
+def test_silu_mul_rejects_too_many_experts(lib):
+    assert lib.ep_silu_mul(FAKE, 4, 256, FAKE, FAKE, 5000, 1, FAKE, FAKE, 0,
+                           None) == B.EP_ERR_UNSUPPORTED
 
 
 def test_binding_raises(lib):
