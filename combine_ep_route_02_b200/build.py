@@ -39,8 +39,21 @@ def _stale() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        glob.glob(os.path.join(CSRC, "*.h")) + [HEADER]
+        glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.c")) + [HEADER]
     return any(os.path.getmtime(d) > t for d in deps)
+
+
+def generate_tables(build_dir: str) -> None:
+    """Writes silu_table.inc (the expert activation's SiLU table) into
+    build_dir with the host generator csrc/gen_silu_table.c."""
+    exe = os.path.join(build_dir, f"gen_silu_table.{os.getpid()}")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-o", exe,
+                           os.path.join(CSRC, "gen_silu_table.c"), "-lm"])
+    out = os.path.join(build_dir, "silu_table.inc")
+    with open(out + ".tmp", "w") as f:
+        subprocess.check_call([exe], stdout=f)
+    os.replace(out + ".tmp", out)
+    os.remove(exe)
 
 
 # Per-file compiler options (none needed at present).
@@ -55,12 +68,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
     os.makedirs(BUILD_DIR, exist_ok=True)
     tag = f"{os.getpid()}"
+    generate_tables(BUILD_DIR)
     procs, objs = [], []
     for src in sources():
         name = os.path.basename(src)
         obj = os.path.join(BUILD_DIR, name[:-3] + f".{tag}.o")
         cmd = [nvcc(), *ARCH, *COMPILE_FLAGS, *PER_FILE.get(name, []), *extra,
-               "-c", src, "-o", obj]
+               "-I", BUILD_DIR, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), file=sys.stderr)

@@ -12,19 +12,22 @@
 //   s = bf16(silu(g)), silu(g) = g / (1 + e^-g) correctly rounded
 //   h = bf16(fp32(s * u))
 //   then the dispatch quantiser on h (quant.cuh).
-// The correctly rounded SiLU takes an fp32 evaluation (expf and a fast
-// divide, a few fp32 ulps of error) and rounds it to bf16 unless the fp32
-// value lies within 64 fp32 ulps of a bf16 rounding midpoint, or g is
-// outside the range where that error bound holds; those inputs take an fp64
-// evaluation.  Every one of the 65,536 bf16 inputs is checked against the
-// oracle on the GPU.
+// The correctly rounded SiLU is a function of the 16-bit gate pattern: a
+// table generated at build time (gen_silu_table.c, x87 extended precision)
+// holds it for the 8,192 gates with 2^-25 <= |g| < 2^7, and each block keeps
+// a copy in shared memory.  Outside that range it has closed forms (below:
+// g/2 with ties toward +inf; above: g for g > 0 and -0 for g < 0), taken only
+// by warps that meet such a gate.  Every one of the 65,536 bf16 gates is
+// checked against the oracle on the GPU.
 //
 // Mapping: the filled rows are numbered v = 0 .. V-1 in expert order (V = sum
-// of the counts); a thread owns a 16-element chunk of one output row (two
-// 16-byte loads of gate, two of up, one 16-byte store of e4m3), and the 8
-// lanes of a 128-element block reduce its amax with shuffles.  Each block
-// keeps the counts' prefix sum in shared memory and finds a chunk's expert
-// by binary search.
+// of the counts) and each block takes a contiguous range of them; a thread
+// owns a 16-element chunk of one output row (two 16-byte loads of gate, two
+// of up, one 16-byte store of e4m3), and the 8 lanes of a 128-element block
+// reduce its amax with shuffles.  Each block keeps the counts' prefix sum in
+// shared memory; a thread finds its first chunk's expert by binary search
+// and then walks forward.  The next chunk's loads are issued before the
+// current chunk is computed.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 #include "quant.cuh"
@@ -35,58 +38,88 @@ namespace {
 
 constexpr int ACT_THREADS = 256;
 
-// bf16 value of silu(g) in the slow cases: NaN, -inf, tiny |g|, g < -80, or
-// an fp32 result too close to a bf16 midpoint.
-__device__ __noinline__ float silu_bf16_slow(float g)
+// silu(g) correctly rounded to bf16 for the gates with 2^-25 <= |g| < 2^7,
+// generated at build time (gen_silu_table.c): entry (sign << 12) | (|g|
+// pattern - 0x3300).
+constexpr uint32_t TAB_BASE = 0x3300u;  // |g| pattern of 2^-25
+constexpr int TAB_SIZE = 8192;
+__device__ const uint16_t kSiluTable[TAB_SIZE] = {
+#include "silu_table.inc"
+};
+
+// silu of both gates of a packed bf16 pair w, as a packed bf16 pair, from
+// the table.  Each 16-bit half is offset with its bit 15 set as a guard, so
+// the subtraction never borrows across halves; a half is in the table's
+// range iff its top four bits come out as 1000.  `bad` gets nonzero bits
+// when a gate is outside the range (its entry is then unrelated).
+EP_DEV uint32_t silu_pair_table(uint32_t w, const uint16_t *tab, uint32_t &bad)
 {
-    if (g != g) return g;
-    if (g == -INFINITY) return -0.0f;
-    if (fabsf(g) < 0x1p-100f) {
-        // silu(g) - g/2 = g tanh(g/2) / 2 > 0, far below fp32 and fp64
-        // resolution here, and g/2 (exact in fp32) can be a bf16 midpoint:
-        // the exact value lies just above g/2, so a tie rounds toward +inf
-        // (up in magnitude for g > 0, down for g < 0).
-        uint32_t u = __float_as_uint(g * 0.5f);
-        u += (u >> 31) ? 0x7FFFu : 0x8000u;
-        return __uint_as_float(u & 0xFFFF0000u);
-    }
-    const double x = (double)g;
-    const double v = x / (1.0 + exp(-x));
-    return __bfloat162float(__double2bfloat16(v));
+    const uint32_t d = ((w & 0x7FFF7FFFu) | 0x80008000u) - TAB_BASE * 0x10001u;
+    bad |= (d & 0xF000F000u) ^ 0x80008000u;
+    const uint32_t i_lo = (d & 0x0FFFu) | ((w >> 3) & 0x1000u);
+    const uint32_t i_hi = ((d >> 16) & 0x0FFFu) | ((w >> 19) & 0x1000u);
+    return __byte_perm((uint32_t)tab[i_lo], (uint32_t)tab[i_hi], 0x5410);
 }
 
-EP_DEV float silu_bf16(float g)
+// silu(g) for any bf16 gate pattern b (low 16 bits), as a bf16 pattern: the
+// table inside its range, else the closed forms.  |g| < 2^-25: silu(g) - g/2
+// = g tanh(g/2) / 2 is positive and below half a bf16 step of g/2, so the
+// result is g/2 (exact in fp32) rounded to bf16 with ties toward +inf (a tie
+// occurs only below 2^-126).  |g| >= 2^7 and inf: g for g > 0, -0 for g < 0
+// (|g e^g| < 2^-180).  NaN: NaN.
+EP_DEV uint32_t silu_any(uint32_t b, const uint16_t *tab)
 {
-    // fast range: e^-g stays below 2^126 (the fast divide's range) and the
-    // quotient stays a normal fp32 number; NaN fails the first comparison
-    if (g >= -80.0f && fabsf(g) >= 0x1p-60f) {
-        const float s = __fdividef(g, 1.0f + expf(-g));
-        const uint32_t u = __float_as_uint(s);
-        // the 16 bits that bf16 rounding drops; 0x8000 is the midpoint
-        if ((u & 0xFFFFu) - (0x8000u - 64u) > 128u) return bf16_lo(pack_bf16x2(s, 0.0f));
+    const uint32_t a = b & 0x7FFFu;
+    if (a - TAB_BASE < 4096u) return tab[((b >> 3) & 0x1000u) | (a - TAB_BASE)];
+    if (a < TAB_BASE) {
+        const uint32_t h = __float_as_uint(__uint_as_float(b << 16) * 0.5f);
+        return ((h + ((h >> 31) ? 0x7FFFu : 0x8000u)) >> 16) & 0xFFFFu;
     }
-    return silu_bf16_slow(g);
+    const bool neg_zero = (b & 0x8000u) && a <= 0x7F80u;
+    return neg_zero ? 0x8000u : b;
 }
 
-// h for the 8 elements of one 16-byte gate vector and one 16-byte up vector
-EP_DEV uint4 silu_mul8(uint4 g, uint4 u)
+// bf16x2 product rounded once to nearest even.  s and u have 8-bit
+// significands, so s * u is exact in fp32 wherever bf16 rounding can give a
+// nonzero result, and this equals bf16(fp32(s * u)).
+EP_DEV uint32_t mul_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// h for the 8 elements of one 16-byte gate vector and one 16-byte up vector.
+// FULL = false: table lookups only, `bad` reports gates the table does not
+// cover (the caller then redoes the chunk with FULL = true).
+template <bool FULL>
+EP_DEV uint4 silu_mul8(uint4 g, uint4 u, const uint16_t *tab, uint32_t &bad)
 {
     const uint32_t gp[4] = {g.x, g.y, g.z, g.w};
     const uint32_t up[4] = {u.x, u.y, u.z, u.w};
     uint32_t h[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        const float lo = __fmul_rn(silu_bf16(bf16_lo(gp[m])), bf16_lo(up[m]));
-        const float hi = __fmul_rn(silu_bf16(bf16_hi(gp[m])), bf16_hi(up[m]));
-        h[m] = pack_bf16x2(lo, hi);
+        const uint32_t s = FULL ? __byte_perm(silu_any(gp[m] & 0xFFFFu, tab),
+                                              silu_any(gp[m] >> 16, tab), 0x5410)
+                                : silu_pair_table(gp[m], tab, bad);
+        h[m] = mul_bf16x2(s, up[m]);
     }
     return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// Filled row number v -> buffer row: the last expert p with cum[p] <= v
-// (experts with no rows share their cum value with the next one and are
-// skipped by taking the last).
-EP_DEV int filled_row(const int *cum, const int *eoff, int P, int v)
+// out of line: only warps that meet a gate outside the table's range call it
+__device__ __noinline__ uint4 silu_mul8_any(uint4 g, uint4 u, const uint16_t *tab)
+{
+    uint32_t unused = 0;
+    return silu_mul8<true>(g, u, tab, unused);
+}
+
+// Filled row number v -> buffer row: expert p is the last one with cum[p] <=
+// v (experts with no rows share their cum value with the next one and are
+// passed over).  A thread's v only grows, so p is found once by binary search
+// and then walked forward.
+EP_DEV int first_expert(const int *cum, int P, int v)
 {
     int lo = 0, hi = P;  // cum[lo] <= v < cum[hi]
     while (hi - lo > 1) {
@@ -94,7 +127,69 @@ EP_DEV int filled_row(const int *cum, const int *eoff, int P, int v)
         if (cum[mid] <= v) lo = mid;
         else hi = mid;
     }
-    return eoff[lo] + (v - cum[lo]);
+    return lo;
+}
+
+EP_DEV int filled_row(const int *cum, const int *eoff, int &p, int v)
+{
+    while (cum[p + 1] <= v) ++p;  // cum[P] = V > v ends the walk
+    return eoff[p] + (v - cum[p]);
+}
+
+// One 16-element chunk in flight: chunk c of buffer row `row`.  A lane whose
+// chunk index is past the block's range (or whose row lies outside the
+// buffer) is inactive and holds zeros: it still takes part in the shuffles
+// but stores nothing (its whole octet is inactive with it).
+struct Chunk {
+    uint4 g0, g1, u0, u1;
+    int row, c;
+    bool active;
+};
+
+EP_DEV void fetch_chunk(Chunk &ch, const uint16_t *__restrict__ gate_up, int n_rows, int I,
+                        const int *cum, const int *eoff, int &p, bool counted, long long base,
+                        long long total, const ChunkWalk &it)
+{
+    ch.g0 = ch.g1 = ch.u0 = ch.u1 = make_uint4(0, 0, 0, 0);
+    ch.row = ch.c = 0;
+    ch.active = base + threadIdx.x < total;
+    if (ch.active) {
+        ch.row = counted ? filled_row(cum, eoff, p, it.t) : it.t;
+        ch.c = it.c;
+        ch.active = (unsigned)ch.row < (unsigned)n_rows;  // offsets beyond the buffer: skipped
+    }
+    if (ch.active) {
+        const uint16_t *gp = gate_up + (size_t)ch.row * 2 * I + (size_t)ch.c * 16;
+        ch.g0 = ld_stream(gp);
+        ch.g1 = ld_stream(gp + 8);
+        ch.u0 = ld_stream(gp + I);
+        ch.u1 = ld_stream(gp + I + 8);
+    }
+}
+
+template <bool FP8>
+EP_DEV void process_chunk(const Chunk &ch, const uint16_t *tab, int I, void *act,
+                          float *act_scale)
+{
+    uint32_t bad = 0;
+    uint4 h0 = silu_mul8<false>(ch.g0, ch.u0, tab, bad);
+    uint4 h1 = silu_mul8<false>(ch.g1, ch.u1, tab, bad);
+    if (__any_sync(FULL_MASK, bad != 0)) {  // rare: a gate below 2^-25 or above 2^7
+        h0 = silu_mul8_any(ch.g0, ch.u0, tab);
+        h1 = silu_mul8_any(ch.g1, ch.u1, tab);
+    }
+    if (FP8) {
+        float scale;
+        const uint4 q = quant::quant_chunk(h0, h1, scale);
+        if (ch.active) {
+            st_stream(static_cast<uint8_t *>(act) + (size_t)ch.row * I + (size_t)ch.c * 16, q);
+            if ((ch.c & 7) == 0) st_stream_f32(act_scale + (size_t)ch.row * (I >> 7) + (ch.c >> 3), scale);
+        }
+    } else if (ch.active) {
+        uint16_t *o = static_cast<uint16_t *>(act) + (size_t)ch.row * I + (size_t)ch.c * 16;
+        st_stream(o, h0);
+        st_stream(o + 8, h1);
+    }
 }
 
 template <bool FP8>
@@ -107,11 +202,17 @@ silu_mul_kernel(const uint16_t *__restrict__ gate_up, int n_rows, int I,
     int *cum = sm;            // [P + 1]  prefix sum of the counts
     int *eoff = sm + P + 1;   // [P]      first buffer row of each expert
     __shared__ int warp_tot[ACT_THREADS / 32 + 1];
+    __shared__ __align__(16) uint16_t tab[TAB_SIZE];
     pdl_launch_dependents();
+    // the table is no input of this call: copy it while the previous kernel
+    // finishes
+    for (int i = threadIdx.x; i < TAB_SIZE / 8; i += blockDim.x)
+        reinterpret_cast<uint4 *>(tab)[i] = reinterpret_cast<const uint4 *>(kSiluTable)[i];
     pdl_wait();
 
     int V = n_rows;
-    if (expert_off != nullptr) {
+    const bool counted = expert_off != nullptr;
+    if (counted) {
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         // block-wide exclusive scan of the counts, ACT_THREADS at a time
         int carry = 0;
@@ -134,48 +235,36 @@ silu_mul_kernel(const uint16_t *__restrict__ gate_up, int n_rows, int I,
             __syncthreads();
         }
         if (threadIdx.x == 0) cum[P] = carry;
-        __syncthreads();
         V = min(carry, n_rows);
     }
+    __syncthreads();  // table and prefix sums complete
 
     const int cpr = I >> 4;        // 16-element chunks per output row (multiple of 8)
-    const int S = I >> 7;
-    const long long total = (long long)V * cpr;
-    const long long stride = (long long)gridDim.x * ACT_THREADS;
-    // block-uniform loop bound so every lane reaches the shuffles; total is
-    // a multiple of 8, so a lane octet is all active or all idle
-    ChunkWalk it((long long)blockIdx.x * ACT_THREADS + threadIdx.x, stride, cpr);
-    for (long long base = (long long)blockIdx.x * ACT_THREADS; base < total;
-         base += stride, it.next()) {
-        bool active = base + threadIdx.x < total;
-        const int c = it.c;
-        int row = 0;
-        uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0, u0 = g0, u1 = g0;
-        if (active) {
-            row = expert_off != nullptr ? filled_row(cum, eoff, P, it.t) : it.t;
-            active = (unsigned)row < (unsigned)n_rows;  // offsets beyond the buffer: skipped
-        }
-        if (active) {
-            const uint16_t *gp = gate_up + (size_t)row * 2 * I + (size_t)c * 16;
-            g0 = ld_stream(gp);
-            g1 = ld_stream(gp + 8);
-            u0 = ld_stream(gp + I);
-            u1 = ld_stream(gp + I + 8);
-        }
-        const uint4 h0 = silu_mul8(g0, u0);
-        const uint4 h1 = silu_mul8(g1, u1);
-        if (FP8) {
-            float scale;
-            const uint4 q = quant::quant_chunk(h0, h1, scale);
-            if (active) {
-                st_stream(static_cast<uint8_t *>(act) + (size_t)row * I + (size_t)c * 16, q);
-                if ((c & 7) == 0) st_stream_f32(act_scale + (size_t)row * S + (c >> 3), scale);
-            }
-        } else if (active) {
-            uint16_t *o = static_cast<uint16_t *>(act) + (size_t)row * I + (size_t)c * 16;
-            st_stream(o, h0);
-            st_stream(o + 8, h1);
-        }
+    // each block takes a contiguous range of filled rows, so a thread's
+    // expert index moves forward by at most one expert per row it crosses
+    const long long rows_per_block = ((long long)V + gridDim.x - 1) / gridDim.x;
+    const long long v0 = min((long long)V, (long long)blockIdx.x * rows_per_block);
+    const long long v1 = min((long long)V, v0 + rows_per_block);
+    const long long total = v1 * cpr;
+    const long long stride = ACT_THREADS;
+    // block-uniform loop bound so every lane reaches the shuffles; the range
+    // starts and ends on row boundaries (cpr is a multiple of 8), so a lane
+    // octet is all active or all idle
+    long long base = v0 * cpr;
+    ChunkWalk it(base + threadIdx.x, stride, cpr);
+    int p = (counted && base + threadIdx.x < total) ? first_expert(cum, P, it.t) : 0;
+    Chunk cur;
+    fetch_chunk(cur, gate_up, n_rows, I, cum, eoff, p, counted, base, total, it);
+    while (base < total) {
+        // issue the next chunk's loads before computing this one
+        ChunkWalk nit = it;
+        nit.next();
+        Chunk nxt;
+        fetch_chunk(nxt, gate_up, n_rows, I, cum, eoff, p, counted, base + stride, total, nit);
+        process_chunk<FP8>(cur, tab, I, act, act_scale);
+        cur = nxt;
+        it = nit;
+        base += stride;
     }
 }
 

@@ -23,10 +23,11 @@ namespace quant {
 EP_DEV float div_by_scale(float x, float scale, float rcp)
 {
     const float q0 = __fmul_rn(x, rcp);
-    const float r = __fmaf_rn(-q0, scale, x);
-    // scale > 0, so the quotient carries the sign of x; the correction
-    // would turn x = -0 into +0 (r = +0, then +0 + -0 = +0)
-    return copysignf(__fmaf_rn(r, rcp, q0), x);
+    // the residual with its sign flipped, q0 * scale - x (exact in one FMA);
+    // adding its negation keeps the sign of a zero quotient: for x = -0 it
+    // gives -0 + -0 = -0, where x - q0 * scale would give +0 + -0 = +0
+    const float rn = __fmaf_rn(q0, scale, -x);
+    return __fmaf_rn(-rn, rcp, q0);
 }
 
 // The correction is exact while the residual cannot underflow: for a
@@ -39,21 +40,26 @@ EP_DEV bool fast_div_ok(float scale)
     return scale >= 0x1p-90f && scale <= 0x1p125f;
 }
 
-EP_DEV uint32_t quant4(const float *v, float scale, float rcp, bool fast)
+// q = e4m3(fp32(x / scale)) for 16 values: FAST divides through the block's
+// reciprocal (normal scales, see fast_div_ok), otherwise by IEEE division.
+// The two are separate code paths so that neither is executed predicated
+// beside the other.
+template <bool FAST>
+EP_DEV uint4 quant16(const float *v, float scale, float rcp)
 {
-    // q = e4m3(fp32(x / scale))
-    float q[4];
+    float q[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = fast ? div_by_scale(v[i], scale, rcp) : __fdiv_rn(v[i], scale);
-    return pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
+    for (int i = 0; i < 16; ++i) q[i] = FAST ? div_by_scale(v[i], scale, rcp) : __fdiv_rn(v[i], scale);
+    uint4 r;
+    r.x = pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
+    r.y = pack_e4m3x2(q[4], q[5]) | (pack_e4m3x2(q[6], q[7]) << 16);
+    r.z = pack_e4m3x2(q[8], q[9]) | (pack_e4m3x2(q[10], q[11]) << 16);
+    r.w = pack_e4m3x2(q[12], q[13]) | (pack_e4m3x2(q[14], q[15]) << 16);
+    return r;
 }
 
-// Quantise one 16-element chunk (two 16-byte bf16 vectors).  The 8 lanes
-// whose chunks form one 128-element block must call this together (xor
-// shuffles over lane offsets 1, 2, 4); every lane of the warp must call it.
-EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
+EP_DEV void unpack16(uint4 lo, uint4 hi, float *v)
 {
-    float v[16];
     v[0] = bf16_lo(lo.x);  v[1] = bf16_hi(lo.x);
     v[2] = bf16_lo(lo.y);  v[3] = bf16_hi(lo.y);
     v[4] = bf16_lo(lo.z);  v[5] = bf16_hi(lo.z);
@@ -62,6 +68,24 @@ EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
     v[10] = bf16_lo(hi.y); v[11] = bf16_hi(hi.y);
     v[12] = bf16_lo(hi.z); v[13] = bf16_hi(hi.z);
     v[14] = bf16_lo(hi.w); v[15] = bf16_hi(hi.w);
+}
+
+// out of line, values passed packed: only blocks with a tiny (or non-finite)
+// scale take it
+static __device__ __noinline__ uint4 quant16_ieee(uint4 lo, uint4 hi, float scale)
+{
+    float v[16];
+    unpack16(lo, hi, v);
+    return quant16<false>(v, scale, 0.0f);
+}
+
+// Quantise one 16-element chunk (two 16-byte bf16 vectors).  The 8 lanes
+// whose chunks form one 128-element block must call this together (xor
+// shuffles over lane offsets 1, 2, 4); every lane of the warp must call it.
+EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
+{
+    float v[16];
+    unpack16(lo, hi, v);
 
     float amax = 0.0f;
 #pragma unroll
@@ -72,16 +96,9 @@ EP_DEV uint4 quant_chunk(uint4 lo, uint4 hi, float &scale_out)
     const float scale = __fdiv_rn(amax, 448.0f);
     scale_out = scale;
 
-    uint4 q = make_uint4(0, 0, 0, 0);  // amax == 0: scale 0, zero bytes
-    if (amax != 0.0f) {
-        const bool fast = fast_div_ok(scale);
-        const float rcp = fast ? __frcp_rn(scale) : 0.0f;
-        q.x = quant4(v + 0, scale, rcp, fast);
-        q.y = quant4(v + 4, scale, rcp, fast);
-        q.z = quant4(v + 8, scale, rcp, fast);
-        q.w = quant4(v + 12, scale, rcp, fast);
-    }
-    return q;
+    if (amax == 0.0f) return make_uint4(0, 0, 0, 0);  // scale 0, zero bytes
+    if (fast_div_ok(scale)) return quant16<true>(v, scale, __frcp_rn(scale));
+    return quant16_ieee(lo, hi, scale);  // scales below 2^-90 (or inf, NaN): rare
 }
 
 }  // namespace quant
