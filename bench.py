@@ -487,6 +487,9 @@ def main():
         act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
         pk, pk_kind = peak_hbm()
         gemm = {"row_align": A, "I": I, "recv_rows_capacity": pa.n_recv,
+                "silu_mul_traffic": profiled_traffic(
+                    "silu_mul_kernel_v3.md", f"{cfg.name} T={cfg.T} I={I} row_align={A}",
+                    ("activation.cu", "quant.cuh", "ep_device.cuh", "ep_internal.h")),
                 "recv_rows_used": used, "padding_rows": used - V,
                 "route_layout_us": rl_a_ms * 1e3,
                 "silu_mul_us": act_ms * 1e3, "silu_mul_gbs": act_gbs,
