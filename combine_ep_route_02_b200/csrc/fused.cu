@@ -15,9 +15,10 @@ namespace ep {
 
 namespace {
 
-// shared memory of the last block: the count / slot phase tables, then a
-// copy of the pair list (count writes it at P + R, slot keeps its own there)
-#define SMALL_SMEM_PAIRS_OFFSET(a) \
+// shared memory of the last block: the count / slot phase tables, then what
+// the count phase hands to the slot phase (the pair list, the expert and
+// rank counts, the status bits), past the end of the slot phase's tables
+#define SMALL_SMEM_READY_OFFSET(a) \
     (2 * (a).P + 1 + (a).hist_warps * (a).P + (a).T * (a).k)
 
 template <int EPL>
@@ -43,14 +44,16 @@ route_layout_small_kernel(RouteArgs r, LayoutArgs a, int vec4, int *done)
     __syncthreads();
     if (!is_last) return;
     __threadfence();  // every other block's top-k is visible to the last block
-    // the whole batch is tile 0; the slot phase reuses the pair list the
-    // count phase built, copied out of its way first
-    int *pairs = smem + SMALL_SMEM_PAIRS_OFFSET(a);
+    // the whole batch is tile 0; the slot phase takes the pair list and the
+    // counts from shared memory, copied out of its way first
+    int *ready = smem + SMALL_SMEM_READY_OFFSET(a);
     layout_impl::count_tile(a, 0, smem, &bad_sh);
     const int npairs = a.T * a.k;
-    for (int i = threadIdx.x; i < npairs; i += blockDim.x) pairs[i] = smem[a.P + a.R + i];
+    for (int i = threadIdx.x; i < npairs; i += blockDim.x) ready[i] = smem[a.P + a.R + i];
+    for (int i = threadIdx.x; i < a.P + a.R; i += blockDim.x) ready[npairs + i] = smem[i];
+    if (threadIdx.x == 0) ready[npairs + a.P + a.R] = bad_sh;
     __syncthreads();
-    layout_impl::slot_tile<256, true>(a, 0, smem, warp_tot, pairs);
+    layout_impl::slot_tile<256, true>(a, 0, smem, warp_tot, ready);
 }
 
 template <int EPL>
@@ -82,10 +85,12 @@ cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *don
     a.n_tiles = 1;
     a.hist_warps = layout_hist_warps(a.P) < 8 ? layout_hist_warps(a.P) : 8;
     const size_t pairs = (size_t)r.T * r.k;
-    const size_t count_ints = (size_t)a.P + a.R + pairs;
+    const size_t count_ints = layout_impl::count_smem_ints(a.P, a.R, r.T, r.k);
     const size_t slot_ints = (size_t)2 * a.P + 1 + (size_t)a.hist_warps * a.P + pairs;
-    // tables of the larger phase, then the copied pair list
-    const size_t smem = sizeof(int) * ((count_ints > slot_ints ? count_ints : slot_ints) + pairs);
+    // tables of the larger phase, then the hand-over region (it starts at
+    // slot_ints, beyond every count-phase table it is copied from)
+    const size_t big = count_ints > slot_ints ? count_ints : slot_ints;
+    const size_t smem = sizeof(int) * (big + pairs + a.P + a.R + 1);
     const int vec4 = (r.E % 4 == 0) && ((reinterpret_cast<uintptr_t>(r.logits) & 15) == 0);
     if (r.E <= 32) return launch_small<1>(r, a, vec4, done, smem, s);
     if (r.E <= 64) return launch_small<2>(r, a, vec4, done, smem, s);

@@ -108,7 +108,7 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
     if (a.T == 0) return launch_pdl(layout_empty_kernel, dim3(1), dim3(256), 0, s, a);
     const int NT = a.n_tiles;
     const size_t pairs = (size_t)a.tile_tokens * a.k;
-    const size_t sm_count = sizeof(int) * ((size_t)a.P + a.R + pairs);
+    const size_t sm_count = sizeof(int) * count_smem_ints(a.P, a.R, a.tile_tokens, a.k);
     const size_t sm_slot =
         sizeof(int) * ((size_t)2 * a.P + 1 + (size_t)a.hist_warps * a.P + pairs);
     const bool fused = NT <= LAYOUT_FUSED_MAX_TILES;

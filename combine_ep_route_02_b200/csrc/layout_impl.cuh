@@ -60,18 +60,30 @@ EP_DEV void fill_pairs(const LayoutArgs &a, int t0, int npairs, int *pp, int *hi
     }
 }
 
-// Counts one tile (the block's threads cooperate; smem: P + R + tile_tokens*k
-// ints, bad_sh: one shared int).  Writes tile_cnt / tile_tok / tile_bad row
-// `tile` and in_rank for the tile's tokens.
+// Shared memory of count_tile, in ints: hist [P], tokr [R], pairs
+// [tile_tokens * k], then (8-byte aligned) the token rank masks [tile_tokens]
+// as 64-bit words.
+inline size_t count_smem_ints(int P, int R, int tile_tokens, int k)
+{
+    return (((size_t)P + R + (size_t)tile_tokens * k + 1) & ~(size_t)1) + 2 * (size_t)tile_tokens;
+}
+
+// Counts one tile (the block's threads cooperate; smem: count_smem_ints
+// ints; bad_sh: one shared int).  Writes tile_cnt / tile_tok / tile_bad row
+// `tile` and in_rank for the tile's tokens; hist and tokr stay in shared
+// memory for a caller that lays the tile out in the same block.
 EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
 {
     int *hist = smem;          // [P]
     int *tokr = hist + a.P;    // [R]
     int *pp = tokr + a.R;      // [tile_tokens * k]
+    unsigned long long *tmask = reinterpret_cast<unsigned long long *>(
+        smem + (((size_t)a.P + a.R + (size_t)a.tile_tokens * a.k + 1) & ~(size_t)1));
     int &bad_sh = *bad_sh_p;
     const int t0 = tile * a.tile_tokens;
     const int nt = min(a.tile_tokens, a.T - t0);
     const int npairs = nt * a.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
 
     for (int i = threadIdx.x; i < a.P; i += blockDim.x) hist[i] = 0;
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) tokr[i] = 0;
@@ -85,21 +97,51 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
 
     const int epr = a.P / a.R;
     if (a.R <= 64) {
-        // thread per token: the set of ranks it reaches as a bit mask, then
-        // its in_rank row byte by byte (consecutive threads write
-        // neighbouring rows)
+        // the set of ranks each token reaches, as a bit mask
         for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
             unsigned long long m = 0;
             for (int j = 0; j < a.k; ++j) {
                 const int p = pp[tl * a.k + j];
                 if (p >= 0) m |= 1ull << (p / epr);
             }
-            uint8_t *row = a.in_rank + (size_t)(t0 + tl) * a.R;
-            for (int r = 0; r < a.R; ++r) row[r] = (uint8_t)((m >> r) & 1ull);
-            while (m) {
-                atomicAdd(&tokr[__ffsll((long long)m) - 1], 1);
-                m &= m - 1;
+            tmask[tl] = m;
+        }
+        __syncthreads();
+        // tokens per rank: a ballot per rank over each warp's 32 tokens,
+        // one shared atomic per (warp, rank)
+        int c_lo = 0, c_hi = 0;  // counts of ranks lane and lane + 32
+        for (int base = warp * 32; base < nt; base += nwarps * 32) {  // warp-uniform
+            const unsigned long long m = base + lane < nt ? tmask[base + lane] : 0ull;
+            for (int r = 0; r < a.R; ++r) {
+                const int c = __popc(__ballot_sync(FULL_MASK, (m >> r) & 1ull));
+                if (r < 32) c_lo += (lane == r) ? c : 0;
+                else c_hi += (lane == r - 32) ? c : 0;
             }
+        }
+        if (lane < a.R && c_lo) atomicAdd(&tokr[lane], c_lo);
+        if (lane + 32 < a.R && c_hi) atomicAdd(&tokr[lane + 32], c_hi);
+        // in_rank rows: the tile's rows are one contiguous byte range;
+        // consecutive threads write consecutive 4-byte words of it
+        uint8_t *dst = a.in_rank + (size_t)t0 * a.R;
+        const int nbytes = nt * a.R;
+        const bool words = (reinterpret_cast<uintptr_t>(dst) & 3) == 0;
+        const int nw = words ? nbytes >> 2 : 0;
+        for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+            int tl = (4 * w) / a.R, r = 4 * w - tl * a.R;
+            uint32_t v = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                v |= (uint32_t)((tmask[tl] >> r) & 1ull) << (8 * q);
+                if (++r == a.R) {
+                    r = 0;
+                    ++tl;
+                }
+            }
+            reinterpret_cast<uint32_t *>(dst)[w] = v;
+        }
+        for (int b = 4 * nw + threadIdx.x; b < nbytes; b += blockDim.x) {
+            const int tl = b / a.R, r = b - tl * a.R;
+            dst[b] = (uint8_t)((tmask[tl] >> r) & 1ull);
         }
     } else {
         for (int i = threadIdx.x; i < nt * a.R; i += blockDim.x) {
@@ -156,10 +198,12 @@ EP_DEV int block_exclusive_scan(int *v, int n, int *warp_tot)
 // tile_tokens*k ints; warp_tot: NTHREADS/32 + 1 shared ints).  Tile 0 also
 // writes the batch-wide outputs.  FUSED: the tile histograms are raw counts
 // and are summed here; otherwise tile_cnt already holds exclusive per-tile
-// offsets and cnt_expert the totals.
+// offsets and cnt_expert the totals.  ready (single-tile batches counted by
+// the same block, in shared memory): the pairs' physical experts [npairs],
+// then the expert counts [P], the rank token counts [R] and the status bits.
 template <int NTHREADS, bool FUSED>
 EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
-                      const int *pp_ready = nullptr)
+                      const int *ready = nullptr)
 {
     constexpr int NWARPS = NTHREADS / 32;
     const int HW = a.hist_warps;
@@ -175,7 +219,13 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
     const int npairs = nt * a.k;
     for (int i = threadIdx.x; i < HW * a.P; i += blockDim.x) whist[i] = 0;
 
-    if (FUSED) {
+    const int *ready_hist = ready != nullptr ? ready + npairs : nullptr;
+    if (FUSED && ready != nullptr) {
+        for (int p = threadIdx.x; p < a.P; p += blockDim.x) {
+            toff[p] = 0;
+            eoff[p] = ready_hist[p];
+        }
+    } else if (FUSED) {
         // per expert: rows in tiles before this one, and in all tiles.  Four
         // consecutive lanes share a column, each summing every fourth tile
         // with four loads in flight, then combine by shuffles.
@@ -217,15 +267,18 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
         }
     }
     int bad = 0;  // reported below from the count kernel's tile status words
-    if (pp_ready != nullptr) {  // the same block counted this tile already
-        for (int i = threadIdx.x; i < npairs; i += blockDim.x) pp[i] = pp_ready[i];
+    if (ready != nullptr) {  // the same block counted this tile already
+        for (int i = threadIdx.x; i < npairs; i += blockDim.x) pp[i] = ready[i];
     } else {
         fill_pairs(a, t0, npairs, pp, nullptr, bad);
     }
     __syncthreads();
 
     if (tile == 0) {
-        if (FUSED) {
+        if (FUSED && ready != nullptr) {
+            for (int p = threadIdx.x; p < a.P; p += blockDim.x) a.cnt_expert[p] = eoff[p];
+            for (int r = threadIdx.x; r < a.R; r += blockDim.x) a.tok_rank[r] = ready_hist[a.P + r];
+        } else if (FUSED) {
             for (int p = threadIdx.x; p < a.P; p += blockDim.x) a.cnt_expert[p] = eoff[p];
             // one warp per rank, lanes over tiles (NT <= 64: two loads each)
             for (int r = warp; r < a.R; r += NWARPS) {
@@ -236,7 +289,9 @@ EP_DEV void slot_tile(const LayoutArgs &a, int tile, int *smem, int *warp_tot,
                 if (lane == 0) a.tok_rank[r] = sum;
             }
         }
-        if (a.dev_status != nullptr && threadIdx.x < 32) {
+        if (a.dev_status != nullptr && ready != nullptr) {
+            if (threadIdx.x == 0) *a.dev_status = ready_hist[a.P + a.R];
+        } else if (a.dev_status != nullptr && threadIdx.x < 32) {
             int st = 0;
             for (int i = threadIdx.x; i < NT; i += 32) st |= a.tile_bad[i];
 #pragma unroll
