@@ -9,7 +9,11 @@
 //
 // A block owns one token at a time (persistent over tokens): it reads the
 // gradient row once, streams the k expert rows, writes the k scaled rows and
-// reduces the k dot products across its warps.
+// reduces the k dot products across its warps.  The block has as many
+// threads (a multiple of 32, at most 256) as give every thread the same
+// number of 8-element chunks of a row (224 for H = 7168), and the kernel is
+// compiled for k <= 8 separately so that its partial sums stay in few
+// registers (three blocks per SM).
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -20,7 +24,8 @@ namespace {
 constexpr int BWD_THREADS = 256;
 constexpr int BWD_WARPS = BWD_THREADS / 32;
 
-__global__ void __launch_bounds__(BWD_THREADS, 2)
+template <int KMAX>
+__global__ void __launch_bounds__(BWD_THREADS, KMAX <= 8 ? 3 : 2)
 combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restrict__ y,
                         const int32_t *__restrict__ slot, const float *__restrict__ w, int T,
                         int H, int k, int n_rows, uint16_t *__restrict__ grad_y,
@@ -32,6 +37,7 @@ combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restri
     pdl_launch_dependents();
     pdl_wait();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nthreads = blockDim.x, nwarps = nthreads >> 5;
     const int cpr = H >> 3;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < k) {
@@ -40,10 +46,10 @@ combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restri
             s_w[threadIdx.x] = __ldg(w + (size_t)t * k + threadIdx.x);
         }
         __syncthreads();
-        float part[MAX_TOPK];
+        float part[KMAX];
 #pragma unroll
-        for (int j = 0; j < MAX_TOPK; ++j) part[j] = 0.0f;
-        for (int c = threadIdx.x; c < cpr; c += BWD_THREADS) {
+        for (int j = 0; j < KMAX; ++j) part[j] = 0.0f;
+        for (int c = threadIdx.x; c < cpr; c += nthreads) {
             const uint4 gv = ld_stream(g + (size_t)t * H + (size_t)c * 8);
             const uint32_t gp[4] = {gv.x, gv.y, gv.z, gv.w};
             float gf[8];
@@ -55,7 +61,7 @@ combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restri
             // eight expert rows at a time: all loads issued before the
             // first store (the stores are compiler barriers)
 #pragma unroll
-            for (int j0 = 0; j0 < MAX_TOPK; j0 += 8) {
+            for (int j0 = 0; j0 < KMAX; j0 += 8) {
                 if (j0 >= k) break;
                 uint4 yv[8];
 #pragma unroll
@@ -88,7 +94,7 @@ combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restri
         }
         // reduce each dot product over the block
 #pragma unroll
-        for (int j = 0; j < MAX_TOPK; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
             if (j >= k) break;
             float v = part[j];
 #pragma unroll
@@ -99,7 +105,7 @@ combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restri
         if (threadIdx.x < k) {
             float v = 0.0f;
 #pragma unroll
-            for (int q = 0; q < BWD_WARPS; ++q) v += s_part[q][threadIdx.x];
+            for (int q = 0; q < nwarps; ++q) v += s_part[q][threadIdx.x];
             grad_w[(size_t)t * k + threadIdx.x] = (s_slot[threadIdx.x] >= 0) ? v : 0.0f;
         }
         __syncthreads();  // s_slot / s_w / s_part are rewritten for the next token
@@ -112,7 +118,18 @@ cudaError_t launch_combine_backward(const CombineBackwardArgs &a, cudaStream_t s
 {
     if (a.T == 0) return cudaSuccess;
     const int blocks = a.T < a.grid ? a.T : a.grid;
-    return launch_pdl(combine_backward_kernel, dim3(blocks), dim3(BWD_THREADS), 0, s,
+    // threads per block: the fewest multiples of 32 (up to BWD_THREADS) that
+    // give every thread the same number of 8-element chunks of a row
+    const int cpr = a.H / 8;
+    const int per = (cpr + BWD_THREADS - 1) / BWD_THREADS;
+    int nt = ((cpr + per - 1) / per + 31) / 32 * 32;
+    if (nt > BWD_THREADS) nt = BWD_THREADS;
+    if (a.k <= 8)
+        return launch_pdl(combine_backward_kernel<8>, dim3(blocks), dim3(nt), 0, s,
+                          static_cast<const uint16_t *>(a.g), static_cast<const uint16_t *>(a.y),
+                          a.slot, a.w, a.T, a.H, a.k, a.n_rows, static_cast<uint16_t *>(a.grad_y),
+                          a.grad_w);
+    return launch_pdl(combine_backward_kernel<MAX_TOPK>, dim3(blocks), dim3(nt), 0, s,
                       static_cast<const uint16_t *>(a.g), static_cast<const uint16_t *>(a.y),
                       a.slot, a.w, a.T, a.H, a.k, a.n_rows, static_cast<uint16_t *>(a.grad_y),
                       a.grad_w);
@@ -121,7 +138,7 @@ cudaError_t launch_combine_backward(const CombineBackwardArgs &a, cudaStream_t s
 int combine_backward_blocks_per_sm()
 {
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_backward_kernel, BWD_THREADS, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_backward_kernel<8>, BWD_THREADS, 0);
     return n > 0 ? n : 1;
 }
 

@@ -52,12 +52,22 @@ EP_DEV void fill_pairs(const LayoutArgs &a, int t0, int npairs, int *pp, int *hi
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u * (int)blockDim.x;
             if (i < npairs) {
-                const int p = phys_of_id(a, t0 + i / a.k, e[u], bad);
+                // the token index only matters for the replica choice
+                const int t = a.phys_of != nullptr ? t0 + i / a.k : 0;
+                const int p = phys_of_id(a, t, e[u], bad);
                 pp[i] = p;
                 if (hist != nullptr && p >= 0) atomicAdd(&hist[p], 1);
             }
         }
     }
+}
+
+// floor(n / d) for 0 <= n < 2^22 and 1 <= d <= 2^22 without an integer
+// division: (n + 1/2) / d lies at least 1/(2d) from the nearest integer, far
+// more than the rounding error of the fp32 product, so truncation is exact.
+EP_DEV int small_div(int n, float inv_d)
+{
+    return __float2int_rz(__fmul_rn((float)n + 0.5f, inv_d));
 }
 
 // Shared memory of count_tile, in ints: hist [P], tokr [R], pairs
@@ -96,13 +106,14 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
     __syncthreads();
 
     const int epr = a.P / a.R;
+    const float inv_epr = 1.0f / (float)epr, inv_R = 1.0f / (float)a.R;
     if (a.R <= 64) {
         // the set of ranks each token reaches, as a bit mask
         for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
             unsigned long long m = 0;
             for (int j = 0; j < a.k; ++j) {
                 const int p = pp[tl * a.k + j];
-                if (p >= 0) m |= 1ull << (p / epr);
+                if (p >= 0) m |= 1ull << small_div(p, inv_epr);
             }
             tmask[tl] = m;
         }
@@ -127,7 +138,7 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
         const bool words = (reinterpret_cast<uintptr_t>(dst) & 3) == 0;
         const int nw = words ? nbytes >> 2 : 0;
         for (int w = threadIdx.x; w < nw; w += blockDim.x) {
-            int tl = (4 * w) / a.R, r = 4 * w - tl * a.R;
+            int tl = small_div(4 * w, inv_R), r = 4 * w - tl * a.R;
             uint32_t v = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -140,7 +151,7 @@ EP_DEV void count_tile(const LayoutArgs &a, int tile, int *smem, int *bad_sh_p)
             reinterpret_cast<uint32_t *>(dst)[w] = v;
         }
         for (int b = 4 * nw + threadIdx.x; b < nbytes; b += blockDim.x) {
-            const int tl = b / a.R, r = b - tl * a.R;
+            const int tl = small_div(b, inv_R), r = b - tl * a.R;
             dst[b] = (uint8_t)((tmask[tl] >> r) & 1ull);
         }
     } else {
