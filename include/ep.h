@@ -45,7 +45,7 @@
  *  - Layout: row-major, densely packed.  Index arrays are int32.
  *  - Errors: argument checks happen on the host before anything is enqueued
  *    and return EP_ERR_INVALID (bad shape / value / alignment) or
- *    EP_ERR_UNSUPPORTED (valid but beyond this build's limits).  A launch
+ *    EP_ERR_UNSUPPORTED (valid but beyond the library's limits).  A launch
  *    failure returns EP_ERR_CUDA.  Bad data found on the device (an expert id
  *    outside [0,E), an invalid replica map entry) never traps: it sets bits
  *    in the caller's *dev_status and the offending pair gets slot -1.
