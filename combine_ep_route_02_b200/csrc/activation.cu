@@ -286,7 +286,10 @@ cudaError_t launch_activation(const ActivationArgs &a, cudaStream_t s)
     const int P = a.expert_off != nullptr ? a.P : 0;
     const size_t smem = act_smem_bytes(P);
     const void *fn = a.fp8 ? (const void *)silu_mul_kernel<true> : (const void *)silu_mul_kernel<false>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // the kernel also holds 16 KB of static shared memory (the SiLU table):
+    // opt in above the default 48 KB for the sum of the two
+    if (smem + sizeof(uint16_t) * TAB_SIZE + 1024 > 48 * 1024)
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     // without counts the work is known on the host: no more blocks than chunks
     long long blocks = a.grid;
     if (a.expert_off == nullptr) {

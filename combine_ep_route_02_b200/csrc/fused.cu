@@ -62,7 +62,9 @@ cudaError_t launch_small(const RouteArgs &r, const LayoutArgs &a, int vec4, int 
 {
     cudaError_t e = cudaMemsetAsync(done, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
-    if (smem > 48 * 1024)
+    // dynamic plus the kernel's static shared memory (under 1 KB) above the
+    // default 48 KB needs an opt-in
+    if (smem + 1024 > 48 * 1024)
         cudaFuncSetAttribute(route_layout_small_kernel<EPL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int blocks = (r.T + 7) / 8;  // a warp per token: T <= SMALL_MAX_PAIRS

@@ -96,7 +96,9 @@ __global__ void layout_empty_kernel(LayoutArgs a)
 
 void opt_in_smem(const void *fn, size_t bytes)
 {
-    if (bytes > 48 * 1024)
+    // dynamic plus the kernels' static shared memory (under 1 KB) above the
+    // default 48 KB needs an opt-in
+    if (bytes + 1024 > 48 * 1024)
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 

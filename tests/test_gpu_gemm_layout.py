@@ -256,3 +256,69 @@ def test_silu_mul_graph_replay_follows_new_counts():
         assert np.array_equal(act.cpu().numpy(), q_ref)
         assert np.array_equal(sc.cpu().numpy(), s_ref)
     del g
+
+
+@pytest.mark.parametrize("T,align", [(700, 1024), (20000, 128)])
+def test_padded_layout_max_sizes(T, align):
+    """P = 4096, k = 32, R = 64, skewed ids, the largest row tile; T = 20000
+    takes the column-scan path"""
+    from combine_ep_route_02_b200 import ep_dispatch_layout, ep_workspace_size
+    rng = np.random.default_rng(12)
+    k, E, R = 32, 4096, 64
+    idx = np.argsort(rng.random((T, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
+    idx[::3, :8] = np.arange(8)
+    ref = oracle.layout(idx, E, E, R, row_align=align)
+    n_src = T * k + E * (align - 1)
+    d = dict(cnt_expert=E, expert_off=E + 1, rows_rank=R, rank_off=R + 1, tok_rank=R,
+             slot=(T, k), src=n_src)
+    g = {n: torch.full(s if isinstance(s, tuple) else (s,), -5, dtype=torch.int32,
+                       device="cuda") for n, s in d.items()}
+    in_rank = torch.empty((T, R), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ep_workspace_size(T, k, E, R), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ep_dispatch_layout(torch.from_numpy(idx).cuda(), T, k, E, E, R, None, None, 0,
+                       g["cnt_expert"], g["expert_off"], g["rows_rank"], g["rank_off"],
+                       g["tok_rank"], in_rank, g["slot"], g["src"], ws, st, row_align=align)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    used = int(ref["expert_off"][-1])
+    for n in d:
+        got = g[n].cpu().numpy()
+        if n == "src":
+            assert np.all(got[used:] == -5)     # beyond the used rows: untouched
+            got = got[:used]
+        assert np.array_equal(got.reshape(ref[n].shape), ref[n]), n
+    assert np.array_equal(in_rank.cpu().numpy(), ref["in_rank"])
+
+
+def test_silu_mul_many_experts_and_gaps():
+    """P = 4096 experts with synthetic counts (many empty), offsets with gaps
+    between experts, and some offsets beyond the buffer: rows past the
+    buffer are skipped, every other counted row matches the oracle"""
+    rng = np.random.default_rng(13)
+    P, I = 4096, 256
+    cnt = rng.integers(0, 4, P).astype(np.int32)
+    cnt[rng.random(P) < 0.5] = 0
+    gaps = rng.integers(0, 3, P)
+    off = np.zeros(P + 1, np.int64)
+    for p in range(P):
+        off[p + 1] = off[p] + cnt[p] + gaps[p]
+    n_rows = int(off[P]) - 50                   # the last experts run past the buffer
+    eo = off.astype(np.int32)
+    gu = oracle.bf16_encode_array(rng.standard_normal((n_rows, 2 * I)).astype(np.float32))
+    q, sc = run_silu(gu, True, eo, cnt, P, 0x5A, -9.0)
+    sent_q = np.full((n_rows, I), 0x5A, np.uint8)
+    sent_s = np.full((n_rows, I // 128), -9.0, np.float32)
+    q_ref, s_ref = oracle.silu_mul_quant(gu, True, eo, cnt, sent_q, sent_s)
+    assert np.array_equal(q, q_ref)
+    assert np.array_equal(sc, s_ref)
+
+
+def test_silu_mul_empty_counts():
+    """all counts zero: nothing is written"""
+    P, I, n = 64, 128, 40
+    eo = np.zeros(P + 1, np.int32)
+    cnt = np.zeros(P, np.int32)
+    gu = np.full((n, 2 * I), 0x3F80, np.uint16)
+    q, sc = run_silu(gu, True, eo, cnt, P, 0x5A, -9.0)
+    assert np.all(q == 0x5A) and np.all(sc == -9.0)
