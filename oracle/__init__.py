@@ -6,7 +6,8 @@ never does.  The arithmetic lives in ``ep_oracle.c`` (plain C, fp32 where the
 method fixes fp32, fp64 for the sigmoid); this file only compiles it and
 marshals numpy arrays.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` against
+Every function here is pinned by ``tests/test_oracle_pins.py`` (and the
+expert activation by ``tests/test_oracle_activation.py``) against
 brute force, closed forms, invariants or a library routine.
 """
 
