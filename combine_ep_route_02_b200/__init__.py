@@ -29,4 +29,6 @@ from ._binding import (  # noqa: F401
     ep_workspace_size,
     lib,
 )
+from .exchange import (ExchangePlan, combine_exchange, dispatch_exchange,  # noqa: F401
+                       exchange_plan)
 from .path import EpHostPipeline, EpMicroBatchPipeline, EpPath  # noqa: F401
