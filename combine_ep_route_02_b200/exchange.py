@@ -64,10 +64,15 @@ def exchange_plan(rows_rank, cnt_expert, group=None) -> ExchangePlan:
     if ce.numel() % world:
         raise ValueError("the number of physical experts must be a multiple of the group size")
     epr = ce.numel() // world
-    # one all-to-all of [rows, count of each local expert] per destination
-    send = torch.cat([rr.view(world, 1), ce.view(world, epr)], dim=1).contiguous()
+    # one all-to-all of [rows, count of each local expert] per destination,
+    # on the device the group's backend works on (NCCL: the current GPU)
+    dev = torch.device("cpu")
+    if dist.get_backend(group) == "nccl":
+        dev = torch.device("cuda", torch.cuda.current_device())
+    send = torch.cat([rr.view(world, 1), ce.view(world, epr)], dim=1).contiguous().to(dev)
     recv = torch.empty_like(send)
     dist.all_to_all_single(recv, send, group=group)
+    recv = recv.cpu()
     return ExchangePlan(send_splits=rr.tolist(), recv_splits=recv[:, 0].tolist(),
                         recv_cnt=recv[:, 1:].clone(), rank=rank, world=world)
 
