@@ -18,6 +18,8 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle
 from gen import CONFIGS, Workload
@@ -600,3 +602,41 @@ def test_layout_row_alignment(align):
     if align == 1:
         for n in ("expert_off", "slot", "src", "rows_rank", "rank_off"):
             assert np.array_equal(lay[n], base[n])
+
+
+def _padded_layout_restatement(idx, E, R, align):
+    """slots by a stable sort of the pairs by expert (pairs in (t, j) order),
+    expert starts rounded up to the row tile"""
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    order = np.argsort(flat, kind="stable")
+    cnt = np.bincount(flat, minlength=E)
+    padded = -(-cnt // align) * align
+    off = np.concatenate([[0], np.cumsum(padded)])
+    first_in_sorted = np.concatenate([[0], np.cumsum(cnt)])
+    slot = np.empty(T * k, np.int64)
+    for pos, pair in enumerate(order):
+        e = flat[pair]
+        slot[pair] = off[e] + (pos - first_in_sorted[e])
+    epr = E // R
+    return cnt, off, slot.reshape(T, k), off[::epr]
+
+
+@settings(max_examples=60, deadline=None)
+@given(T=st.integers(1, 40), k=st.integers(1, 4), epr=st.integers(1, 4), R=st.integers(1, 4),
+       align=st.sampled_from([1, 2, 3, 8, 16]), seed=st.integers(0, 2 ** 31 - 1))
+def test_padded_layout_vs_sort_restatement(T, k, epr, R, align, seed):
+    E = epr * R
+    if k > E:
+        k = E
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    lay = oracle.layout(idx, E, E, R, row_align=align)
+    cnt, off, slot, rank_off = _padded_layout_restatement(idx, E, R, align)
+    assert np.array_equal(lay["cnt_expert"], cnt)
+    assert np.array_equal(lay["expert_off"], off)
+    assert np.array_equal(lay["slot"], slot)
+    assert np.array_equal(lay["rank_off"], rank_off)
+    src = np.full(off[-1], -1)
+    src[slot.reshape(-1)] = np.arange(T * k)
+    assert np.array_equal(lay["src"], src)
