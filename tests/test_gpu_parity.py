@@ -602,3 +602,28 @@ def test_combine_backward(name):
     err = np.abs(gw.cpu().numpy().astype(np.float64) - ref_w)
     assert (err <= 1e-5 * mag + 1e-6).all(), float((err - 1e-5 * mag).max())
     assert (gw.cpu().numpy()[~valid] == 0).all()
+
+
+@pytest.mark.parametrize("T,R", [(300, 128), (5000, 256)])
+def test_layout_many_ranks(T, R):
+    """more than 64 logical ranks: in_rank and the rank counts come from the
+    per-(token, rank) path of the count phase"""
+    from combine_ep_route_02_b200 import ep_dispatch_layout, ep_workspace_size
+    rng = np.random.default_rng(14)
+    k, E = 8, 512
+    idx = np.argsort(rng.random((T, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
+    ref = oracle.layout(idx, E, E, R)
+    d = dict(cnt_expert=E, expert_off=E + 1, rows_rank=R, rank_off=R + 1, tok_rank=R,
+             slot=(T, k), src=T * k)
+    g = {n: torch.empty(s, dtype=torch.int32, device="cuda") for n, s in d.items()}
+    in_rank = torch.empty((T, R), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ep_workspace_size(T, k, E, R), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ep_dispatch_layout(torch.from_numpy(idx).cuda(), T, k, E, E, R, None, None, 0,
+                       g["cnt_expert"], g["expert_off"], g["rows_rank"], g["rank_off"],
+                       g["tok_rank"], in_rank, g["slot"], g["src"], ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for n in d:
+        assert np.array_equal(g[n].cpu().numpy().reshape(ref[n].shape), ref[n]), n
+    assert np.array_equal(in_rank.cpu().numpy(), ref["in_rank"])
