@@ -627,3 +627,33 @@ def test_layout_many_ranks(T, R):
     for n in d:
         assert np.array_equal(g[n].cpu().numpy().reshape(ref[n].shape), ref[n]), n
     assert np.array_equal(in_rank.cpu().numpy(), ref["in_rank"])
+
+
+@pytest.mark.parametrize("k,H", [(12, 2048), (32, 1024), (3, 7168)])
+def test_combine_backward_topk_and_widths(k, H):
+    """top-k above 8 (the general instance of the kernel) and row widths that
+    give different block sizes"""
+    from combine_ep_route_02_b200 import ep_combine_backward
+    rng = np.random.default_rng(k * 100 + H)
+    T = 97
+    n = T * k
+    slot = rng.permutation(n).astype(np.int32).reshape(T, k)
+    slot[5, k - 1] = -1
+    w = rng.uniform(0.05, 1.5, (T, k)).astype(np.float32)
+    y = device_normal_bf16(n, H, seed=k)
+    g = device_normal_bf16(T, H, seed=k + 1)
+    gy = torch.zeros((n, H), dtype=torch.bfloat16, device="cuda")
+    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ep_combine_backward(g, y, torch.from_numpy(slot).cuda(), torch.from_numpy(w).cuda(), T, H, k,
+                        gy, gw)
+    torch.cuda.synchronize()
+    ref_y, ref_w = oracle.combine_backward(g.cpu(), y.cpu(), slot, w)
+    assert np.array_equal(u16(gy), ref_y)
+    yc, gc = y.cpu().double().numpy(), g.cpu().double().numpy()
+    valid = slot >= 0
+    mag = np.zeros_like(ref_w, dtype=np.float64)
+    mag[valid] = np.einsum("th,th->t", np.abs(gc)[np.nonzero(valid)[0]],
+                           np.abs(yc[slot[valid]]))
+    err = np.abs(gw.cpu().numpy().astype(np.float64) - ref_w)
+    assert (err <= 1e-5 * mag + 1e-6).all()
+    assert (gw.cpu().numpy()[~valid] == 0).all()
