@@ -21,11 +21,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_batch(rank, align):
+def _rank_batch(rank, align, world=2):
     """this rank's layout and FP8 receive rows (recomputable from the seed)"""
     import oracle
     from gen import CONFIGS, Workload
-    cfg = dataclasses.replace(CONFIGS["ds16b"].scaled(96), R=2)
+    E = 64 if world == 2 else 48
+    cfg = dataclasses.replace(CONFIGS["ds16b"].scaled(96), R=world, E=E)
     wl = Workload(cfg, seed=1000 + rank)
     idx, w, _ = oracle.route(wl.logits, wl.bias, cfg.n_group, cfg.topk_group, cfg.topk,
                              cfg.routed_scale, cfg.renorm)
@@ -54,7 +55,7 @@ def _rank_main(rank, world, port, align, out_dir):
         sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
         from combine_ep_route_02_b200.exchange import (combine_exchange, dispatch_exchange,
                                                        exchange_plan)
-        cfg, lay, rx, rs, _ = _rank_batch(rank, align)
+        cfg, lay, rx, rs, _ = _rank_batch(rank, align, world)
         plan = exchange_plan(lay["rows_rank"], lay["cnt_expert"])
         got_x = dispatch_exchange(torch.from_numpy(rx), plan)
         got_s = dispatch_exchange(torch.from_numpy(rs), plan)
@@ -71,12 +72,11 @@ def _rank_main(rank, world, port, align, out_dir):
         dist.destroy_process_group()
 
 
-def _check(tmp_path, align):
-    world = 2
+def _check(tmp_path, align, world=2):
     port = _free_port()
     mp.start_processes(_rank_main, args=(world, port, align, str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
-    batches = [_rank_batch(r, align) for r in range(world)]
+    batches = [_rank_batch(r, align, world) for r in range(world)]
     for me in range(world):
         res = np.load(tmp_path / f"rank{me}.npz")
         parts_x, parts_s, cnts = [], [], []
@@ -103,3 +103,7 @@ def test_exchange_two_ranks(tmp_path):
 
 def test_exchange_two_ranks_gemm_layout(tmp_path):
     _check(tmp_path, 16)
+
+
+def test_exchange_three_ranks(tmp_path):
+    _check(tmp_path, 8, world=3)
