@@ -71,39 +71,6 @@ def tokens_per_s(T: int, world: int, steps: int, max_ms: float) -> float:
     return T * world * steps / (max_ms * 1e-3)
 
 
-def kernel_source_hash(*names) -> str:
-    """sha256 over the given kernel source files (package csrc/)."""
-    import hashlib
-    h = hashlib.sha256()
-    for n in names:
-        with open(os.path.join(ROOT, "combine_ep_route_02_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()
-
-
-def profiled_traffic(summary: str, workload: str, sources):
-    """DRAM bytes per launch recorded in profiles/<summary> for this
-    workload, or None when the kernel's sources changed since the capture."""
-    path = os.path.join(ROOT, "profiles", summary)
-    try:
-        text = open(path).read()
-    except OSError:
-        return None
-    fields = {}
-    for line in text.splitlines():
-        if line.startswith("- ") and ":" in line:
-            key, _, val = line[2:].partition(":")
-            fields[key.strip()] = val.strip().strip("`")
-    if fields.get("workload") != workload:
-        return None
-    if fields.get("source_sha256") != kernel_source_hash(*sources):
-        return None
-    try:
-        return int(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
-
-
 def peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -181,21 +148,84 @@ class ClockSampler:
                 "window": window}
 
 
-def cpu_oracle_sample(cfg, wl, y_host_rows, n_tok):
-    """Oracle route+layout+dispatch+combine on the first n_tok tokens."""
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(cfg, wl, y_host_rows, n_tok, threads=1):
+    """Oracle route+layout+dispatch+combine on the first n_tok tokens; with
+    threads > 1 routing, dispatch and combine run token ranges on that many
+    host threads (the layout's counting sweep stays on one)."""
     import oracle
     sub = cfg.scaled(n_tok)
     lg = wl.logits[:n_tok].numpy()
     x = wl.x_rows(0, n_tok)
     t0 = time.perf_counter()
     idx, w, _ = oracle.route(lg, wl.bias, sub.n_group, sub.topk_group, sub.topk,
-                             sub.routed_scale, sub.renorm)
+                             sub.routed_scale, sub.renorm, threads=threads)
     po = None if wl.phys_of is None else wl.phys_of.numpy()
     nr = None if wl.n_rep is None else wl.n_rep.numpy()
     lay = oracle.layout(idx, sub.E, sub.n_phys, sub.R, po, nr)
-    oracle.dispatch(x, lay["slot"], sub.fp8)
-    oracle.combine(y_host_rows, lay["slot"], w)
+    oracle.dispatch(x, lay["slot"], sub.fp8, threads=threads)
+    oracle.combine(y_host_rows, lay["slot"], w, threads=threads)
     return time.perf_counter() - t0
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_replicas(n: int, argv) -> int:
+    """Runs this script as n ranks under torch.distributed.run on this node
+    (one process per GPU, rendezvous on 127.0.0.1) and returns their exit
+    status.  Used when --gpus N > 1 is given without a launcher."""
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_dry(args, cfg):
+    """The multi-rank host logic without a GPU: gloo process group, each rank
+    runs the oracle over a small sample of its own batch (seed = rank) as its
+    step, the slowest rank's time is the job's, rank 0 prints the line."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    n_tok = min(cfg.T, 32)
+    wl = Workload(cfg, seed=rank_seed(rank))
+    g = torch.Generator().manual_seed(rank)
+    y = torch.randn((n_tok * cfg.topk, cfg.H), generator=g).to(torch.bfloat16)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(cfg, wl, y, n_tok)
+    secs = sum(cpu_oracle_sample(cfg, wl, y, n_tok) for _ in range(args.steps))
+    max_ms = reduce_max(secs * 1e3, dist, "cpu")
+    if rank == 0:
+        value = tokens_per_s(n_tok, world, args.steps, max_ms)
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "host oracle (dry run)", "data": "synthetic", "dry_run": True,
+            "config": {"workload": cfg.name, "T": n_tok, "H": cfg.H, "E": cfg.E,
+                       "topk": cfg.topk, "parallelism": f"replicas x{world}",
+                       "note": "no GPU: each rank's step is the CPU oracle on its own batch"}}),
+            flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_reference(args, cfg):
@@ -207,9 +237,10 @@ def run_reference(args, cfg):
     wl = Workload(cfg)
     g = torch.Generator().manual_seed(7)
     y = torch.randn((n_tok * cfg.topk, cfg.H), generator=g).to(torch.bfloat16)
+    cores = host_cores()
     for _ in range(args.warmup):
-        cpu_oracle_sample(cfg, wl, y, n_tok)
-    times = [cpu_oracle_sample(cfg, wl, y, n_tok) for _ in range(args.steps)]
+        cpu_oracle_sample(cfg, wl, y, n_tok, threads=cores)
+    times = [cpu_oracle_sample(cfg, wl, y, n_tok, threads=cores) for _ in range(args.steps)]
     tot = sum(times)
     value = n_tok * args.steps / tot
     line = {
@@ -220,8 +251,9 @@ def run_reference(args, cfg):
         "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "topk": cfg.topk,
                    "sample_tokens": n_tok},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {n_tok} of {cfg.T} tokens per step, single thread"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {n_tok} of {cfg.T} tokens per step, routing, "
+                                   f"dispatch and combine split over {cores} host threads"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -256,7 +288,12 @@ def main():
                     help="skip timing the GEMM layout (padded rows) and the expert activation")
     ap.add_argument("--row-align", type=int, default=128,
                     help="row tile of the GEMM layout timed after the step")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="no GPU: check the multi-rank launch, the max-over-ranks timing and "
+                         "the output line with gloo ranks running the CPU oracle")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_replicas(args.gpus, sys.argv[1:]))
     faulthandler.enable()
     cfg = CONFIGS[args.config]
     if args.tokens > 0:
@@ -266,6 +303,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, cfg)
+        return
+    if args.dry_run:
+        run_dry(args, cfg)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -332,14 +372,21 @@ def main():
     t_wall0 = time.perf_counter()
 
     # 1. eager launches on one stream, events around route+layout, dispatch
-    #    and combine (the per-kernel attribution and the roofline)
+    #    and combine (the per-kernel attribution and the roofline); a batch
+    #    small enough for the one-kernel route+layout+dispatch runs that
+    #    kernel between s0 and d1 (d0 is recorded just before it)
+    fused = path.fused_route_dispatch()
     for i in range(K):
         if flush:
             flush_l2(i)  # evict the previous step's data from L2
         s0[i].record(stream)
-        path.route_layout(lg, bias)
-        d0[i].record(stream)
-        path.dispatch(x)
+        if fused:
+            d0[i].record(stream)
+            path.route_dispatch(lg, bias, x)
+        else:
+            path.route_layout(lg, bias)
+            d0[i].record(stream)
+            path.dispatch(x)
         d1[i].record(stream)
         c0[i].record(stream)
         path.combine(y)
@@ -487,9 +534,6 @@ def main():
         act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
         pk, pk_kind = peak_hbm()
         gemm = {"row_align": A, "I": I, "recv_rows_capacity": pa.n_recv,
-                "silu_mul_traffic": profiled_traffic(
-                    "silu_mul_kernel_v3.md", f"{cfg.name} T={cfg.T} I={I} row_align={A}",
-                    ("activation.cu", "quant.cuh", "ep_device.cuh", "ep_internal.h")),
                 "recv_rows_used": used, "padding_rows": used - V,
                 "route_layout_us": rl_a_ms * 1e3,
                 "silu_mul_us": act_ms * 1e3, "silu_mul_gbs": act_gbs,
@@ -508,26 +552,43 @@ def main():
     if True:
         comb_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(c0, c1))
         disp_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(d0, d1))
-        comb_gbs = ab["combine"] / (comb_ms * 1e-3) / 1e9
-        disp_gbs = ab["dispatch"] / (disp_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "combine_kernel", "achieved": comb_gbs,
-                    "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
-                    "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy)"
-                    if peak_kind == "measured" else "fallback 6650 GB/s",
-                    "traffic": profiled_traffic(
-                        "combine_kernel_v3.md", f"{cfg.name} T={cfg.T}",
-                        ("combine.cu", "ep_device.cuh", "ep_internal.h"))}
-        dc_ms = comb_ms + disp_ms
         rl_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(s0, d0))
+        comb_gbs = ab["combine"] / (comb_ms * 1e-3) / 1e9
+        # the fused kernel moves the routing, layout and dispatch bytes
+        disp_bytes = ab["dispatch"] + (ab["route"] + ab["layout"] if fused else 0)
+        disp_gbs = disp_bytes / (disp_ms * 1e-3) / 1e9
+        peak_src = (f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy)" if peak_kind == "measured"
+                    else "fallback 6650 GB/s")
+        # the dominant kernel of the step by event time
+        if comb_ms >= disp_ms:
+            dom, dom_gbs, dom_bytes, dom_ms = "combine_kernel", comb_gbs, ab["combine"], comb_ms
+        else:
+            dom = ("route_dispatch_small_kernel" if fused else "dispatch_fp8_tma_kernel"
+                   if cfg.fp8 else "dispatch_bf16_kernel")
+            dom_gbs, dom_bytes, dom_ms = disp_gbs, disp_bytes, disp_ms
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": dom_gbs,
+                    "peak": peak, "unit": "GB/s", "frac": dom_gbs / peak,
+                    "peak_source": peak_src,
+                    "algorithmic_bytes_per_launch": dom_bytes,
+                    "launch_us": dom_ms * 1e3,
+                    "timing": "CUDA events on the launching stream around each launch, "
+                              "mean over the K eager steps",
+                    # DRAM bytes need a profiler's counters, which this run does
+                    # not collect; the ncu captures are kept with the profiles
+                    "traffic": None}
+        dc_ms = comb_ms + disp_ms
         extra = {
-            "route_layout_us": rl_ms * 1e3,
-            "dispatch_us": disp_ms * 1e3, "combine_us": comb_ms * 1e3,
+            "route_layout_us": None if fused else rl_ms * 1e3,
+            "dispatch_us": None if fused else disp_ms * 1e3,
+            "route_dispatch_us": disp_ms * 1e3 if fused else None,
+            "combine_us": comb_ms * 1e3,
             "dispatch_gbs": disp_gbs, "combine_gbs": comb_gbs,
             "dispatch_combine_tokens_per_s": cfg.T * world / (dc_ms * 1e-3),
             "dispatch_combine_gbs": (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3) / 1e9,
             "dispatch_combine_frac_of_peak": (ab["dispatch"] + ab["combine"]) / (dc_ms * 1e-3)
             / 1e9 / peak,
             "step_gbs": step_bytes / (tot_ms / K * 1e-3) / 1e9,
+            "step_us": tot_ms / K * 1e3,
         }
 
     # end to end through the public API: every step uploads its inputs from
@@ -560,16 +621,28 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # whole passes of the oracle over the workload's batch until about
-        # 10 s of CPU work (at most 8 passes)
+        # whole passes of the oracle over the workload's batch, on one thread
+        # and then on every host core, until about 10 s of CPU work each (at
+        # most 8 passes)
         yh = y.cpu()
-        secs, passes = 0.0, 0
-        while passes < 8 and (secs < 10.0 or passes == 0):
-            secs += cpu_oracle_sample(cfg, wl, yh, cfg.T)
-            passes += 1
-        cpu = {"value": cfg.T * passes / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{passes} pass(es) of route+layout+dispatch+combine over all "
-                         f"{cfg.T} tokens of the same batch, single thread ({secs:.1f} s)"}
+        cores = host_cores()
+
+        def oracle_rate(threads):
+            secs, passes = 0.0, 0
+            while passes < 8 and (secs < 10.0 or passes == 0):
+                secs += cpu_oracle_sample(cfg, wl, yh, cfg.T, threads=threads)
+                passes += 1
+            return cfg.T * passes / secs, passes, secs
+
+        v1, p1, s1_ = oracle_rate(1)
+        vn, pn, sn = oracle_rate(cores)
+        cpu = {"value": vn, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{pn} pass(es) of route+layout+dispatch+combine over all {cfg.T} "
+                         f"tokens of the same batch, routing, dispatch and combine split "
+                         f"over {cores} host threads ({sn:.1f} s)",
+               "single_thread": {"value": v1, "cores": 1,
+                                 "sample": f"{p1} pass(es) over all {cfg.T} tokens, one "
+                                           f"thread ({s1_:.1f} s)"}}
 
     if rank == 0:
         line = {
@@ -582,7 +655,8 @@ def main():
                        "P": cfg.n_phys, "R": cfg.R, "n_group": cfg.n_group,
                        "topk_group": cfg.topk_group, "topk": cfg.topk, "fp8": cfg.fp8,
                        "routed_scale": cfg.routed_scale, "cuda_graph": micro_ms is None,
-                       "l2": ("flushed before each step (256 MiB write, outside step events)"
+                       "l2": ("flushed before each step (256 MiB written, then another "
+                              "256 MiB read, outside the step's events)"
                               if flush else
                               f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB moved per step)"),
                        "parallelism": f"replicas x{world}",

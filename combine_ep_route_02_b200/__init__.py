@@ -10,6 +10,7 @@ call does, and raises if it has not been built.
 from ._binding import (  # noqa: F401
     EP_DEV_BAD_EXPERT,
     EP_DEV_BAD_REPLICA,
+    EP_DEV_TIMEOUT,
     EP_ERR_CUDA,
     EP_ERR_DEVICE,
     EP_ERR_INVALID,
@@ -24,7 +25,9 @@ from ._binding import (  # noqa: F401
     ep_dispatch,
     ep_dispatch_layout,
     ep_route,
+    ep_route_dispatch,
     ep_route_layout,
+    ep_testing_set_wait_limit,
     ep_silu_mul,
     ep_workspace_size,
     lib,

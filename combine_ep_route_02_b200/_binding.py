@@ -25,10 +25,11 @@ EP_DEV_BAD_EXPERT = 1
 EP_DEV_BAD_REPLICA = 2
 EP_DEV_TIMEOUT = 4
 
-# every symbol declared in include/ep.h
+# every symbol declared in include/ep.h and include/ep_testing.h
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
            "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout",
-           "ep_dispatch_backward", "ep_combine_backward", "ep_silu_mul")
+           "ep_dispatch_backward", "ep_combine_backward", "ep_silu_mul", "ep_route_dispatch",
+           "ep_testing_set_wait_limit")
 
 
 class EpError(RuntimeError):
@@ -77,6 +78,11 @@ def lib() -> ctypes.CDLL:
         L.ep_combine_backward.restype = I
         L.ep_silu_mul.argtypes = [P, I, I, P, P, I, I, P, P, I, P]
         L.ep_silu_mul.restype = I
+        L.ep_route_dispatch.argtypes = [P, P, I, RouteCfg, I, I, P, P, I, I, P, I, I, I, P, P,
+                                        P, P, P, P, P, P, P, P, P, P, P, I, P, P]
+        L.ep_route_dispatch.restype = I
+        L.ep_testing_set_wait_limit.argtypes = [ctypes.c_longlong]
+        L.ep_testing_set_wait_limit.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -161,6 +167,25 @@ def ep_route_layout(logits, bias, T, cfg: RouteCfg, P, R, phys_of, n_rep, max_re
         _ptr(topk_idx), _ptr(topk_w), _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank),
         _ptr(rank_off), _ptr(tok_rank), _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace),
         _ptr(dev_status), _stream(stream)))
+
+
+def ep_route_dispatch(logits, bias, T, cfg: RouteCfg, P, R, phys_of, n_rep, max_rep, x, H, fp8,
+                      recv_x, recv_scale, topk_idx, topk_w, cnt_expert, expert_off, rows_rank,
+                      rank_off, tok_rank, in_rank, slot, src, workspace, dev_status, stream=None,
+                      *, row_align=1, recv_rows=0, num_sms=0):
+    """ep_route_layout followed by ep_dispatch (one kernel for small batches)."""
+    _check("ep_route_dispatch", lib().ep_route_dispatch(
+        _ptr(logits), _ptr(bias), T, cfg, P, R, _ptr(phys_of), _ptr(n_rep), max_rep, row_align,
+        _ptr(x), H, int(bool(fp8)), recv_rows, _ptr(recv_x), _ptr(recv_scale), _ptr(topk_idx),
+        _ptr(topk_w), _ptr(cnt_expert), _ptr(expert_off), _ptr(rows_rank), _ptr(rank_off),
+        _ptr(tok_rank), _ptr(in_rank), _ptr(slot), _ptr(src), _ptr(workspace), num_sms,
+        _ptr(dev_status), _stream(stream)))
+
+
+def ep_testing_set_wait_limit(polls: int):
+    """Failure-detection tests only: polls of every bounded device wait in
+    later launches (0 = give up at once, negative = the default)."""
+    _check("ep_testing_set_wait_limit", lib().ep_testing_set_wait_limit(int(polls)))
 
 
 def ep_dispatch_backward(grad_recv, slot, T, H, k, grad_x, num_sms=0, dev_status=None,

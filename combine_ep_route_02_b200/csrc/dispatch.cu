@@ -99,8 +99,7 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
 // ---------------------------------------------------------------------------
 constexpr int TMA_IN_STAGES = 4;
 constexpr int TMA_OUT_STAGES = 4;
-constexpr uint32_t TMA_WAIT_LIMIT = 1u << 22;  // polls before reporting a timeout
-constexpr int DEV_TIMEOUT = 4;                 // EP_DEV_TIMEOUT
+constexpr int DEV_TIMEOUT = 4;  // EP_DEV_TIMEOUT
 
 __host__ __device__ inline size_t tma_smem_bytes(int H)
 {
@@ -111,7 +110,8 @@ __host__ __device__ inline size_t tma_smem_bytes(int H)
 __global__ void __launch_bounds__(512)
 dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                         const int32_t *__restrict__ slot, uint8_t *__restrict__ recv_x,
-                        float *__restrict__ recv_scale, int n_rows, int32_t *dev_status)
+                        float *__restrict__ recv_scale, int n_rows, int32_t *dev_status,
+                        uint32_t wait_limit)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int S = H >> 7;
@@ -147,7 +147,7 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
         const int o = it % TMA_OUT_STAGES;
         int my_slot = -1;
         if (warp == 0 && lane < k) my_slot = __ldg(slot + (size_t)t * k + lane);
-        const bool ok = mbar_wait(bar_base + 8 * st, (it / TMA_IN_STAGES) & 1, TMA_WAIT_LIMIT);
+        const bool ok = mbar_wait(bar_base + 8 * st, (it / TMA_IN_STAGES) & 1, wait_limit);
         if (!__syncthreads_and(ok)) {
             failed_at = it;
             break;
@@ -198,9 +198,11 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
     if (warp == 0 && lane < k) bulk_wait_all();
     if (failed_at >= 0 && tid == 0) {
         // let the loads still in flight land before the CTA's shared memory
-        // goes away, then report
+        // goes away (with the default limit, whatever limit gave up), then
+        // report
         for (int it = failed_at; it < n_my && it < failed_at + TMA_IN_STAGES; ++it)
-            mbar_wait(bar_base + 8 * (it % TMA_IN_STAGES), (it / TMA_IN_STAGES) & 1, TMA_WAIT_LIMIT);
+            mbar_wait(bar_base + 8 * (it % TMA_IN_STAGES), (it / TMA_IN_STAGES) & 1,
+                      WAIT_LIMIT_DEFAULT);
         if (dev_status != nullptr) atomicOr(dev_status, DEV_TIMEOUT);
     }
 }
@@ -249,7 +251,7 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s)
         return launch_pdl(dispatch_fp8_tma_kernel, dim3(blocks), dim3(tma_threads(a.H)),
                           tma_smem_bytes(a.H), s, static_cast<const uint16_t *>(a.x), a.T, a.H,
                           a.k, a.slot, static_cast<uint8_t *>(a.recv_x), a.recv_scale,
-                          a.n_rows, a.dev_status);
+                          a.n_rows, a.dev_status, a.wait_limit);
     }
     const long long chunks = (long long)a.T * (a.fp8 ? a.H / 16 : a.H / 8);
     long long blocks = (chunks + DISPATCH_THREADS - 1) / DISPATCH_THREADS;

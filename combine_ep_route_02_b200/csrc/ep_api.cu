@@ -1,9 +1,22 @@
 // C-ABI entry points of libep_b200: host-side argument checks, launch
 // configuration, and the mapping of CUDA errors to ep_status.
+#include <atomic>
+
 #include "../../include/ep.h"
+#include "../../include/ep_testing.h"
 #include "ep_internal.h"
 
 namespace ep {
+
+namespace {
+std::atomic<long long> g_wait_limit{-1};  // < 0: the default
+}  // namespace
+
+uint32_t wait_limit()
+{
+    const long long v = g_wait_limit.load(std::memory_order_relaxed);
+    return v < 0 ? WAIT_LIMIT_DEFAULT : (uint32_t)v;
+}
 
 int device_sm_count()
 {
@@ -226,9 +239,61 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
         return EP_ERR_INVALID;
     DispatchArgs a{x_bf16, T, H, k, slot, fp8 != 0, recv_x, recv_scale,
                    streaming_grid(num_sms, cached_blocks_per_sm(fp8 != 0)), 0, dev_status,
-                   rows_of(recv_rows, T, k)};
+                   rows_of(recv_rows, T, k), wait_limit()};
     if (T > 0 && dispatch_tma_ok(a)) a.tma_grid = streaming_grid(num_sms, tma_blocks_per_sm(H));
     return from_cuda(launch_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_route_dispatch(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                            int P, int R, const int32_t *phys_of, const int32_t *n_rep,
+                            int max_rep, int row_align, const void *x_bf16, int H, int fp8,
+                            int recv_rows, void *recv_x, float *recv_scale, int32_t *topk_idx,
+                            float *topk_w, int32_t *cnt_expert, int32_t *expert_off,
+                            int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                            uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
+                            int num_sms, int32_t *dev_status, ep_stream_t stream)
+{
+    ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
+    if (st != EP_OK) return st;
+    const int E = cfg.num_experts, k = cfg.topk;
+    st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align, cnt_expert,
+                      expert_off, rows_rank, rank_off, tok_rank, in_rank, slot, src, workspace,
+                      dev_status);
+    if (st != EP_OK) return st;
+    if (H < 1 || (fp8 ? (H % 128 != 0) : (H % 8 != 0))) return EP_ERR_INVALID;
+    if (T > (1 << 30)) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!x_bf16 || !recv_x || (fp8 && !recv_scale))) return EP_ERR_INVALID;
+    if (!aligned(x_bf16, 16) || !aligned(recv_x, 16) || !aligned(recv_scale, 4))
+        return EP_ERR_INVALID;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int n_rows = rows_of(recv_rows, T, k);
+    const int sms_all = device_sm_count();
+    const int sms = (num_sms <= 0 || num_sms > sms_all) ? sms_all : num_sms;
+    if (small_route_dispatch_ok(T, k, P, H, fp8 != 0, sms)) {
+        const RouteArgs r{logits, bias, T, E, cfg.n_group, cfg.topk_group, k, cfg.routed_scale,
+                          cfg.renorm != 0, topk_idx, topk_w};
+        const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
+                                         row_align, cnt_expert, expert_off, rows_rank, rank_off,
+                                         tok_rank, in_rank, slot, src, workspace, dev_status);
+        int *ctrl = reinterpret_cast<int *>(static_cast<char *>(workspace) +
+                                            layout_workspace_core(T, k, P, R));
+        return from_cuda(launch_route_dispatch_small(r, a, x_bf16, H, fp8 != 0, n_rows, recv_x,
+                                                     recv_scale, sms, ctrl, wait_limit(), s));
+    }
+    // larger batches: the two calls' kernels back to back
+    st = ep_route_layout(logits, bias, T, cfg, P, R, phys_of, n_rep, max_rep, row_align, topk_idx,
+                         topk_w, cnt_expert, expert_off, rows_rank, rank_off, tok_rank, in_rank,
+                         slot, src, workspace, dev_status, stream);
+    if (st != EP_OK) return st;
+    return ep_dispatch(x_bf16, T, H, k, n_rows, slot, fp8, recv_x, recv_scale, num_sms,
+                       dev_status, stream);
+}
+
+ep_status ep_testing_set_wait_limit(long long polls)
+{
+    if (polls > 0xffffffffLL) return EP_ERR_INVALID;
+    g_wait_limit.store(polls < 0 ? -1 : polls, std::memory_order_relaxed);
+    return EP_OK;
 }
 
 ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_w, int T, int H,

@@ -22,6 +22,14 @@ constexpr int MAX_TOPK = 32;
 constexpr int MAX_GROUPS = 32;
 constexpr int MAX_ROW_ALIGN = 1024;  // GEMM row tile of the padded layout
 
+// Polls a bounded device-side wait makes before it gives up and reports
+// EP_DEV_TIMEOUT (a wait for a TMA copy, or for the other blocks of a grid).
+// wait_limit() is this default unless a failure-detection test changed it
+// (ep_testing_set_wait_limit); waits that drain copies still in flight after
+// a give-up always use the default.
+constexpr uint32_t WAIT_LIMIT_DEFAULT = 1u << 22;
+uint32_t wait_limit();
+
 struct RouteArgs {
     const float *logits;
     const float *bias;
@@ -62,6 +70,7 @@ struct DispatchArgs {
     int tma_grid;      // > 0: use the TMA pipeline with this many CTAs
     int32_t *dev_status;
     int n_rows;        // receive rows; slots outside [0, n_rows) are skipped
+    uint32_t wait_limit;  // polls of each bounded TMA wait
 };
 
 struct CombineArgs {
@@ -173,6 +182,12 @@ cudaError_t launch_route(const RouteArgs &a, cudaStream_t s);
 bool small_route_layout_ok(int T, int k, int P);
 cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *done,
                                       cudaStream_t s);
+// Fused routing + layout + dispatch for small batches (one kernel; see
+// decode.cu).  ctrl: 4 ints of workspace (zeroed by the launch).
+bool small_route_dispatch_ok(int T, int k, int P, int H, int fp8, int sms);
+cudaError_t launch_route_dispatch_small(const RouteArgs &r, LayoutArgs a, const void *x, int H,
+                                        int fp8, int n_rows, void *recv_x, float *recv_scale,
+                                        int sms, int *ctrl, uint32_t wait_limit, cudaStream_t s);
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);

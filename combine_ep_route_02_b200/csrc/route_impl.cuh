@@ -72,8 +72,12 @@ EP_DEV double exp_table(double y, const double *tab)
     const double K = 0x1.71547652b82fep+6;   // 64 / ln 2
     const double L1 = 0x1.62e42fefa0000p-7;  // high 36 bits of ln2 / 64
     const double L2 = 0x1.cf79abc9e3b3ap-46; // ln2 / 64 - L1
-    const double Nd = rint(y * K);
-    const int N = (int)Nd;
+    // N = y * K rounded to the nearest integer (ties to even): adding
+    // 1.5 * 2^52 leaves N in the low bits of the sum, since |y K| < 2^51
+    const double SHIFT = 0x1.8p52;
+    const double big = __dadd_rn(__dmul_rn(y, K), SHIFT);
+    const double Nd = __dsub_rn(big, SHIFT);
+    const int N = __double2loint(big);
     double r = fma(-Nd, L1, y);
     r = fma(-Nd, L2, r);
     double p = fma(r, 1.0 / 720.0, 1.0 / 120.0);

@@ -93,6 +93,19 @@ class EpPath:
                           self.tok_rank, self.in_rank, self.slot, self.src, self.workspace,
                           self.dev_status, stream, row_align=self.row_align)
 
+    def route_dispatch(self, logits: torch.Tensor, bias: Optional[torch.Tensor], x: torch.Tensor,
+                       stream=None):
+        """route, layout and dispatch in one call (one kernel for small
+        batches); the same outputs as route_layout then dispatch.  The one
+        dev_status word of the call lands in ``dev_status``."""
+        B.ep_route_dispatch(logits, bias, self.T, self.cfg, self.P, self.R, self.phys_of,
+                            self.n_rep, self.max_rep, x, self.H, self.fp8, self.recv_x,
+                            self.recv_scale, self.topk_idx, self.topk_w, self.cnt_expert,
+                            self.expert_off, self.rows_rank, self.rank_off, self.tok_rank,
+                            self.in_rank, self.slot, self.src, self.workspace, self.dev_status,
+                            stream, row_align=self.row_align, recv_rows=self.n_recv,
+                            num_sms=self.dispatch_sms)
+
     def dispatch(self, x: torch.Tensor, stream=None):
         B.ep_dispatch(x, self.T, self.H, self.k, self.slot, self.fp8, self.recv_x,
                       self.recv_scale, self.dispatch_sms, self.copy_status, stream,
@@ -116,10 +129,27 @@ class EpPath:
                       act_scale is not None, act, act_scale, self.num_sms, stream)
 
     def step(self, x, logits, bias, y, stream=None, out=None):
-        """route, layout, dispatch, then combine of the expert outputs y."""
-        self.route_layout(logits, bias, stream)
-        self.dispatch(x, stream)
+        """route, layout, dispatch (one call), then combine of the expert
+        outputs y."""
+        self.route_dispatch(logits, bias, x, stream)
         return self.combine(y, stream, out)
+
+    def fused_route_dispatch(self) -> bool:
+        """Whether route_dispatch runs as one kernel (mirrors the library's
+        rule: T*k <= 4096, P <= 1024, at most 8 tokens per SM, the block's
+        rows within one TMA transaction and 200 KB of shared memory)."""
+        T, k, P, H = self.T, self.k, self.P, self.H
+        if T <= 0 or T * k > 4096 or P > 1024:
+            return False
+        sms = torch.cuda.get_device_properties(self.recv_x.device).multi_processor_count
+        if self.dispatch_sms > 0:
+            sms = min(sms, self.dispatch_sms)
+        tpb = -(-T // sms)
+        if tpb > 8 or tpb * 2 * H >= 1 << 20:
+            return False
+        xb = tpb * 2 * H + (tpb * H + tpb * (H // 128) * 4 if self.fp8 else 0)
+        xb = (xb + 15) // 16 * 16
+        return xb + 4 * (3 * P + 1 + T * k) <= 200 * 1024
 
     def kernels_per_step(self) -> int:
         """Kernels one step launches: route, layout (count + slot, plus a
@@ -128,6 +158,8 @@ class EpPath:
         tiles can grow, capped by the slot kernel's shared memory)."""
         if self.T == 0:
             return 1
+        if self.fused_route_dispatch():
+            return 2  # route + layout + dispatch in one kernel, combine
         if self.T * self.k <= 4096 and self.P <= 1024:
             return 3  # fused route + layout, dispatch, combine
         tt = max(64, min(512, -(-self.T // 64)))

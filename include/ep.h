@@ -72,7 +72,8 @@ typedef enum {
 /* Bits reported through a caller's *dev_status word. */
 #define EP_DEV_BAD_EXPERT 1  /* layout: a topk_idx entry outside [0, E) */
 #define EP_DEV_BAD_REPLICA 2 /* layout: n_rep[e] outside [1, max_rep] or phys id outside [0, P) */
-#define EP_DEV_TIMEOUT 4     /* dispatch / combine: a bounded wait for an asynchronous copy
+#define EP_DEV_TIMEOUT 4     /* dispatch / route_dispatch: a bounded wait (for an
+                                asynchronous copy, or for the other blocks of the grid)
                                 gave up; that call's output is incomplete */
 
 /* Same object as cudaStream_t; no CUDA header is needed to use this API. */
@@ -210,6 +211,45 @@ ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_rout
 ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
                       const int32_t *slot, int fp8, void *recv_x, float *recv_scale, int num_sms,
                       int32_t *dev_status, ep_stream_t stream);
+
+/*
+ * Routing, dispatch layout and dispatch in one call: the low-latency decode
+ * path of the DeepEP V2 summary (section "Usage for training, prefill and
+ * decoding"), whose small batches are bound by launches and dependency
+ * latency rather than bytes.  Arguments are those of ep_route_layout
+ * followed by those of ep_dispatch (x_bf16, H, fp8, recv_rows, recv_x,
+ * recv_scale), with E = cfg.num_experts and k = cfg.topk; every output is
+ * identical to calling ep_route_layout and then ep_dispatch.  The layout
+ * outputs can be reused by later ep_dispatch / ep_combine calls (the cached
+ * handle of the same section).
+ *
+ * For small batches (T * k <= 4096, P <= 1024, at most 8 tokens per SM and
+ * the rows of a block within 200 KB of shared memory) one kernel does all
+ * three steps with at most one block per SM: each block loads its tokens'
+ * rows with TMA, routes them, quantises them while the other blocks route,
+ * waits at a grid-wide counter in the workspace (a bounded wait), lays out
+ * the whole batch from the T*k ids in L2 and sends its rows to their
+ * receive rows.  Larger batches run ep_route_layout's and ep_dispatch's
+ * kernels back to back.
+ *
+ *   num_sms     SMs to use (0 = all): caps the fused kernel's blocks and the
+ *               dispatch grid
+ *   workspace   ep_workspace_size(T, k, P, R) bytes, 256-byte aligned; need
+ *               not be zeroed (the call clears the words it counts on)
+ *   dev_status  int32 [1] or NULL: zeroed by this call, then the layout's
+ *               EP_DEV_BAD_* bits and EP_DEV_TIMEOUT if a bounded wait (for a
+ *               TMA copy or for the other blocks) gave up, in which case the
+ *               outputs are incomplete
+ * Checks and limits are those of ep_route_layout and ep_dispatch.
+ */
+ep_status ep_route_dispatch(const float *logits, const float *bias, int T, ep_route_cfg cfg,
+                            int P, int R, const int32_t *phys_of, const int32_t *n_rep,
+                            int max_rep, int row_align, const void *x_bf16, int H, int fp8,
+                            int recv_rows, void *recv_x, float *recv_scale, int32_t *topk_idx,
+                            float *topk_w, int32_t *cnt_expert, int32_t *expert_off,
+                            int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank,
+                            uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
+                            int num_sms, int32_t *dev_status, ep_stream_t stream);
 
 /*
  * Combine: weighted gather-reduce back to token order.

@@ -113,6 +113,29 @@ def _ptr(a):
     return None if a is None else a.ctypes.data
 
 
+def _token_ranges(T: int, threads: int):
+    """[t0, t1) ranges splitting T tokens over ``threads`` workers."""
+    n = max(1, min(int(threads), T)) if T > 0 else 1
+    per = -(-T // n) if T > 0 else 0
+    return [(t0, min(T, t0 + per)) for t0 in range(0, T, per)] if T > 0 else []
+
+
+def _run_ranges(fn, T: int, threads: int):
+    """Runs fn(t0, t1) over token ranges, on ``threads`` host threads when
+    more than one (ctypes releases the GIL for the C call, and tokens are
+    independent in routing, dispatch and combine, so each range writes its
+    own outputs).  The arithmetic per token is unchanged."""
+    ranges = _token_ranges(T, threads)
+    if threads <= 1 or len(ranges) <= 1:
+        for r in ranges:
+            fn(*r)
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=len(ranges)) as ex:
+        for f in [ex.submit(fn, *r) for r in ranges]:
+            f.result()
+
+
 def sigmoid(x: float):
     """(fp32 sigmoid, hard flag) for one fp32 input."""
     h = ctypes.c_int(0)
@@ -121,16 +144,22 @@ def sigmoid(x: float):
 
 
 def route(logits, bias, n_group: int, topk_group: int, topk: int,
-          routed_scale: float, renorm: bool):
-    """Returns (topk_idx int32 [T,k], topk_w fp32 [T,k], hard uint8 [T])."""
+          routed_scale: float, renorm: bool, threads: int = 1):
+    """Returns (topk_idx int32 [T,k], topk_w fp32 [T,k], hard uint8 [T]).
+    threads > 1 routes token ranges on that many host threads."""
     lg = _np(logits, np.float32)
     T, E = lg.shape
     b = _np(bias, np.float32)
     idx = np.zeros((T, topk), dtype=np.int32)
     w = np.zeros((T, topk), dtype=np.float32)
     hard = np.zeros(T, dtype=np.uint8)
-    lib().orc_route(_ptr(lg), _ptr(b), T, E, n_group, topk_group, topk,
-                    float(routed_scale), int(bool(renorm)), _ptr(idx), _ptr(w), _ptr(hard))
+    L = lib()
+
+    def part(t0, t1):
+        L.orc_route(_ptr(lg[t0:t1]), _ptr(b), t1 - t0, E, n_group, topk_group, topk,
+                    float(routed_scale), int(bool(renorm)), _ptr(idx[t0:t1]), _ptr(w[t0:t1]),
+                    _ptr(hard[t0:t1]))
+    _run_ranges(part, T, threads)
     return idx, w, hard
 
 
@@ -169,8 +198,10 @@ def quantize_row(x_row):
     return q, sc
 
 
-def dispatch(x, slot, fp8: bool, n_rows=None):
-    """Returns (recv_x, recv_scale); recv_x uint8 [n_rows,H] (fp8) or uint16."""
+def dispatch(x, slot, fp8: bool, n_rows=None, threads: int = 1):
+    """Returns (recv_x, recv_scale); recv_x uint8 [n_rows,H] (fp8) or uint16.
+    threads > 1 dispatches token ranges on that many host threads (the
+    ranges write disjoint receive rows: slots are distinct)."""
     xs = _np(x, np.uint16)
     T, H = xs.shape
     sl = _np(slot, np.int32)
@@ -182,19 +213,30 @@ def dispatch(x, slot, fp8: bool, n_rows=None):
     else:
         rx = np.zeros((n, H), np.uint16)
         rs = None
-    lib().orc_dispatch(_ptr(xs), T, H, k, _ptr(sl), n, int(bool(fp8)), _ptr(rx), _ptr(rs))
+    L = lib()
+
+    def part(t0, t1):
+        L.orc_dispatch(_ptr(xs[t0:t1]), t1 - t0, H, k, _ptr(sl[t0:t1]), n, int(bool(fp8)),
+                       _ptr(rx), _ptr(rs))
+    _run_ranges(part, T, threads)
     return rx, rs
 
 
-def combine(y, slot, topk_w):
-    """out bf16 bits (uint16 [T,H]) = sum_j w * y[slot], fp32 in j order."""
+def combine(y, slot, topk_w, threads: int = 1):
+    """out bf16 bits (uint16 [T,H]) = sum_j w * y[slot], fp32 in j order.
+    threads > 1 combines token ranges on that many host threads."""
     ys = _np(y, np.uint16)
     n, H = ys.shape
     sl = _np(slot, np.int32)
     T, k = sl.shape
     w = _np(topk_w, np.float32)
     out = np.zeros((T, H), np.uint16)
-    lib().orc_combine(_ptr(ys), n, _ptr(sl), _ptr(w), T, H, k, _ptr(out))
+    L = lib()
+
+    def part(t0, t1):
+        L.orc_combine(_ptr(ys), n, _ptr(sl[t0:t1]), _ptr(w[t0:t1]), t1 - t0, H, k,
+                      _ptr(out[t0:t1]))
+    _run_ranges(part, T, threads)
     return out
 
 

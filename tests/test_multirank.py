@@ -74,3 +74,28 @@ def test_replicas_gloo(tmp_path, world):
     lay = oracle.layout(idx, cfg.E, cfg.E, cfg.R)
     rx, rs = oracle.dispatch(wl.x, lay["slot"], True)
     assert float(np.float64(rx.sum()) + np.float64(rs.astype(np.float64).sum())) == digests[1]
+
+
+def test_bench_launches_replicas_itself():
+    """``bench.py --gpus 2`` without a launcher starts two ranks itself
+    (torch.distributed.run on 127.0.0.1); with --dry-run they use gloo and
+    the CPU oracle, and rank 0 alone prints one line for the whole job"""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--dry-run", "--steps", "2", "--warmup", "3", "--config", "tiny"],
+                         capture_output=True, text=True, timeout=600, env=env, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2
+    assert rec["config"]["parallelism"] == "replicas x2"
+    assert rec["scaling"] == "weak" and rec["dry_run"] is True
+    # value = tokens of both ranks over the slowest rank's time
+    assert rec["value"] == pytest.approx(
+        rec["config"]["T"] * 2 * rec["steps"] / (rec["ms_per_step"] * rec["steps"] * 1e-3))
