@@ -29,7 +29,8 @@ EP_DEV_TIMEOUT = 4
 EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
            "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout",
            "ep_dispatch_backward", "ep_combine_backward", "ep_silu_mul", "ep_route_dispatch",
-           "ep_testing_set_wait_limit")
+           "ep_testing_set_wait_limit", "ep_exchange_counts", "ep_dispatch_exchange",
+           "ep_combine_exchange")
 
 
 class EpError(RuntimeError):
@@ -83,6 +84,12 @@ def lib() -> ctypes.CDLL:
         L.ep_route_dispatch.restype = I
         L.ep_testing_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.ep_testing_set_wait_limit.restype = I
+        L.ep_exchange_counts.argtypes = [P, P, P, I, P, P, P]
+        L.ep_exchange_counts.restype = I
+        L.ep_dispatch_exchange.argtypes = [P, P, P, P, Z, P, P]
+        L.ep_dispatch_exchange.restype = I
+        L.ep_combine_exchange.argtypes = [P, P, P, P, Z, P, P]
+        L.ep_combine_exchange.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -186,6 +193,36 @@ def ep_testing_set_wait_limit(polls: int):
     """Failure-detection tests only: polls of every bounded device wait in
     later launches (0 = give up at once, negative = the default)."""
     _check("ep_testing_set_wait_limit", lib().ep_testing_set_wait_limit(int(polls)))
+
+
+def _host_i32(counts):
+    """host int32 array (kept alive by the caller) of a list of counts"""
+    import numpy as np
+    return np.ascontiguousarray(np.asarray(counts, dtype=np.int32))
+
+
+def ep_exchange_counts(comm: int, rows_rank, cnt_expert, P, send_scratch, recv_counts,
+                       stream=None):
+    """comm: the ncclComm_t (an integer address) of a NCCL process group."""
+    _check("ep_exchange_counts", lib().ep_exchange_counts(
+        comm, _ptr(rows_rank), _ptr(cnt_expert), P, _ptr(send_scratch), _ptr(recv_counts),
+        _stream(stream)))
+
+
+def ep_dispatch_exchange(comm: int, rows, send_rows, recv_rows, row_bytes: int, recv,
+                         stream=None):
+    """send_rows / recv_rows: host counts per rank (lists or arrays)."""
+    s, r = _host_i32(send_rows), _host_i32(recv_rows)
+    _check("ep_dispatch_exchange", lib().ep_dispatch_exchange(
+        comm, _ptr(rows), s.ctypes.data, r.ctypes.data, row_bytes, _ptr(recv), _stream(stream)))
+
+
+def ep_combine_exchange(comm: int, expert_rows, recv_rows, send_rows, row_bytes: int, back,
+                        stream=None):
+    s, r = _host_i32(send_rows), _host_i32(recv_rows)
+    _check("ep_combine_exchange", lib().ep_combine_exchange(
+        comm, _ptr(expert_rows), r.ctypes.data, s.ctypes.data, row_bytes, _ptr(back),
+        _stream(stream)))
 
 
 def ep_dispatch_backward(grad_recv, slot, T, H, k, grad_x, num_sms=0, dev_status=None,

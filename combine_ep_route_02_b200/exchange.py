@@ -11,12 +11,17 @@ already writes each destination's rows contiguously, so each direction is one
 all-to-all-v of whole rows, and the combine runs locally on the rows that
 come back in their original order.
 
-The split sizes are the layout's ``rows_rank``; torch.distributed takes them
-as host integers, so building an ``ExchangePlan`` copies ``rows_rank`` and
-``cnt_expert`` to the host once per layout (the handle of the DeepEP V2
-summary is reused for the combine direction).  Rows travel as raw bytes, so
-e4m3 codes, fp32 scales and bf16 rows use the same calls.  With NCCL the
-all-to-all runs over NVLink; with gloo it runs on CPU tensors.
+The split sizes are the layout's ``rows_rank``; they are needed as host
+integers, so building an ``ExchangePlan`` copies the counts to the host once
+per layout (the handle of the DeepEP V2 summary is reused for the combine
+direction).  Rows travel as raw bytes, so e4m3 codes, fp32 scales and bf16
+rows use the same calls.
+
+In a NCCL process group every step runs in the C library on the group's own
+communicator (``ep_exchange_counts``, ``ep_dispatch_exchange``,
+``ep_combine_exchange``: grouped NCCL sends and receives, over NVLink between
+GPUs); this module only marshals arguments.  Other backends (gloo, CPU
+tensors) take torch.distributed's all-to-all with the same split sizes.
 """
 
 from __future__ import annotations
@@ -48,6 +53,25 @@ def _host_ints(t) -> torch.Tensor:
     return torch.as_tensor(t).detach().to("cpu", torch.int64).reshape(-1)
 
 
+_COMM_READY = set()
+
+
+def _nccl_comm(group) -> Optional[int]:
+    """The ncclComm_t (as an integer) behind a NCCL process group on the
+    current device, or None for another backend."""
+    if dist.get_backend(group) != "nccl":
+        return None
+    pg = group if group is not None else dist.distributed_c10d._get_default_group()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    key = (id(pg), dev.index)
+    if key not in _COMM_READY:
+        # the group creates its communicator lazily, at its first collective
+        dist.all_reduce(torch.zeros(1, device=dev), group=group)
+        torch.cuda.synchronize(dev)
+        _COMM_READY.add(key)
+    return int(pg._get_backend(dev)._comm_ptr())
+
+
 def exchange_plan(rows_rank, cnt_expert, group=None) -> ExchangePlan:
     """Exchanges the per-destination row counts and per-expert pair counts.
 
@@ -64,15 +88,23 @@ def exchange_plan(rows_rank, cnt_expert, group=None) -> ExchangePlan:
     if ce.numel() % world:
         raise ValueError("the number of physical experts must be a multiple of the group size")
     epr = ce.numel() // world
-    # one all-to-all of [rows, count of each local expert] per destination,
-    # on the device the group's backend works on (NCCL: the current GPU)
-    dev = torch.device("cpu")
-    if dist.get_backend(group) == "nccl":
+    comm = _nccl_comm(group)
+    if comm is not None:
+        # the counts' all-to-all in the library, on the group's communicator;
+        # then the one device-to-host read of the layout
+        from . import _binding as B
         dev = torch.device("cuda", torch.cuda.current_device())
-    send = torch.cat([rr.view(world, 1), ce.view(world, epr)], dim=1).contiguous().to(dev)
-    recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
-    recv = recv.cpu()
+        rr_d = torch.as_tensor(rows_rank).to(dev, torch.int32).contiguous()
+        ce_d = torch.as_tensor(cnt_expert).to(dev, torch.int32).contiguous()
+        send = torch.empty((world, 1 + epr), dtype=torch.int32, device=dev)
+        recv = torch.empty_like(send)
+        B.ep_exchange_counts(comm, rr_d, ce_d, ce.numel(), send, recv)
+        recv = recv.cpu().to(torch.int64)
+    else:
+        # one all-to-all of [rows, count of each local expert] per destination
+        send = torch.cat([rr.view(world, 1), ce.view(world, epr)], dim=1).contiguous()
+        recv = torch.empty_like(send)
+        dist.all_to_all_single(recv, send, group=group)
     return ExchangePlan(send_splits=rr.tolist(), recv_splits=recv[:, 0].tolist(),
                         recv_cnt=recv[:, 1:].clone(), rank=rank, world=world)
 
@@ -107,9 +139,15 @@ def dispatch_exchange(send_rows: torch.Tensor, plan: ExchangePlan, group=None,
     if out is None:
         out = torch.empty((n_recv,) + tuple(send_rows.shape[1:]), dtype=send_rows.dtype,
                           device=send_rows.device)
-    dist.all_to_all_single(_as_bytes(out[:n_recv], True), _as_bytes(send_rows[:n_send]),
-                           output_split_sizes=plan.recv_splits,
-                           input_split_sizes=plan.send_splits, group=group)
+    dst, src = _as_bytes(out[:n_recv], True), _as_bytes(send_rows[:n_send])
+    comm = _nccl_comm(group)
+    if comm is not None:
+        from . import _binding as B
+        B.ep_dispatch_exchange(comm, src, plan.send_splits, plan.recv_splits,
+                               _row_bytes(send_rows), dst)
+    else:
+        dist.all_to_all_single(dst, src, output_split_sizes=plan.recv_splits,
+                               input_split_sizes=plan.send_splits, group=group)
     return out
 
 
@@ -126,7 +164,13 @@ def combine_exchange(expert_rows: torch.Tensor, plan: ExchangePlan, group=None,
     if out is None:
         out = torch.empty((n_send,) + tuple(expert_rows.shape[1:]), dtype=expert_rows.dtype,
                           device=expert_rows.device)
-    dist.all_to_all_single(_as_bytes(out[:n_send], True), _as_bytes(expert_rows[:n_recv]),
-                           output_split_sizes=plan.send_splits,
-                           input_split_sizes=plan.recv_splits, group=group)
+    dst, src = _as_bytes(out[:n_send], True), _as_bytes(expert_rows[:n_recv])
+    comm = _nccl_comm(group)
+    if comm is not None:
+        from . import _binding as B
+        B.ep_combine_exchange(comm, src, plan.recv_splits, plan.send_splits,
+                              _row_bytes(expert_rows), dst)
+    else:
+        dist.all_to_all_single(dst, src, output_split_sizes=plan.send_splits,
+                               input_split_sizes=plan.recv_splits, group=group)
     return out

@@ -65,7 +65,7 @@ typedef enum {
     EP_OK = 0,
     EP_ERR_INVALID = 1,     /* bad argument: shape, value, alignment, NULL */
     EP_ERR_UNSUPPORTED = 2, /* valid but above a limit of this library */
-    EP_ERR_CUDA = 3,        /* a CUDA launch or API call failed */
+    EP_ERR_CUDA = 3,        /* a CUDA launch or API call (or a NCCL call) failed */
     EP_ERR_DEVICE = 4       /* reserved for callers mapping *dev_status */
 } ep_status;
 
@@ -283,8 +283,10 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
  * ep_workspace_size(T, k, P, R) exceeds that limit return
  * EP_ERR_UNSUPPORTED (with k = 8, P = 256 and R = 8 that is about 2M tokens).
  * The first call on each device looks up the array's device address (host
- * code cannot use the array's name as a device pointer); make that first
- * call before any stream capture.  The call allocates and frees nothing.
+ * code cannot use the array's name as a device pointer) and keeps it for the
+ * life of the process; make that first call before any stream capture.  The
+ * kept address does not survive cudaDeviceReset: after a reset of a device,
+ * do not call this entry point on it again in the same process.  The call allocates and frees nothing.
  * All calls on a device share the one array and it keeps the last call's
  * contents (the kernels need none of them cleared): calls whose work can
  * overlap on the GPU (different streams, or several host threads) race on
@@ -359,6 +361,72 @@ ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, con
 ep_status ep_silu_mul(const void *gate_up_bf16, int n_rows, int I, const int32_t *expert_off,
                       const int32_t *cnt_expert, int P, int fp8, void *act, float *act_scale,
                       int num_sms, ep_stream_t stream);
+
+/*
+ * Expert parallelism across processes (one GPU each) over NCCL: the dispatch
+ * and combine all-to-alls of the Perplexity blog (section "Expert
+ * Parallelism") as grouped NCCL sends and receives of whole rows.  Process
+ * rank q of the communicator is expert-parallel rank q: it owns physical
+ * experts [q*P/W, (q+1)*P/W), so the layout of every rank is computed with
+ * R = W, and rows [rank_off[q], rank_off[q+1]) of its receive buffer are the
+ * ones rank q needs.
+ *
+ * The communicator is the caller's (NCCL's ncclComm_t, for example the one
+ * behind a torch.distributed NCCL process group); the work is enqueued on
+ * `stream`, and the calls must be made in the same order on every rank.  The
+ * library loads NCCL at run time: the NCCL already loaded in the process is
+ * used, and EP_ERR_UNSUPPORTED is returned when none can be loaded.  A NCCL
+ * call that fails returns EP_ERR_CUDA.  Nothing is allocated.
+ *
+ * The row counts of the data exchanges are host integers (NCCL takes its
+ * sizes on the host), so one layout costs one device-to-host read: after
+ * ep_exchange_counts the caller copies recv_counts (and its own rows_rank)
+ * to the host and synchronises the stream, then both directions of the
+ * exchange reuse those counts.
+ */
+typedef struct ncclComm *ep_nccl_comm; /* the same object as NCCL's ncclComm_t */
+
+/*
+ * Counts of one layout's exchange.  Rank q is sent [rows_rank[q],
+ * cnt_expert[q*epr], ..., cnt_expert[q*epr + epr-1]] (epr = P/W), and every
+ * rank's message arrives in recv_counts:
+ *   rows_rank     int32 [W] this rank's receive rows per destination rank
+ *   cnt_expert    int32 [P] this rank's pairs per physical expert
+ *   send_scratch  int32 [W, 1 + P/W] device scratch (the packed messages)
+ *   recv_counts   int32 [W, 1 + P/W] (out): row s = [rows rank s sends
+ *                 here, pairs from s for each of this rank's experts]
+ * P must be a multiple of the communicator's size W.
+ */
+ep_status ep_exchange_counts(ep_nccl_comm comm, const int32_t *rows_rank,
+                             const int32_t *cnt_expert, int P, int32_t *send_scratch,
+                             int32_t *recv_counts, ep_stream_t stream);
+
+/*
+ * Dispatch exchange: rows [sum_{q'<q} send_rows[q'], ... + send_rows[q]) of
+ * `rows` go to rank q, and the recv_rows[s] rows from rank s land in `recv`
+ * starting at row sum_{s'<s} recv_rows[s'] (in the order the source's
+ * layout gave them: by expert, then token).  Rows are row_bytes bytes each,
+ * so the e4m3 codes, their fp32 scale rows and BF16 rows all use this call.
+ *   send_rows  host int32 [W]: this rank's rows_rank
+ *   recv_rows  host int32 [W]: column 0 of recv_counts
+ * The rank's own share is copied on the device; send_rows[me] must equal
+ * recv_rows[me].
+ */
+ep_status ep_dispatch_exchange(ep_nccl_comm comm, const void *rows, const int32_t *send_rows,
+                               const int32_t *recv_rows, size_t row_bytes, void *recv,
+                               ep_stream_t stream);
+
+/*
+ * Combine exchange, the reverse of ep_dispatch_exchange: the expert outputs
+ * of the rows that came from rank s (rows [sum_{s'<s} recv_rows[s'], ... +
+ * recv_rows[s]) of expert_rows) go back to rank s, and the rows returning
+ * from rank q land in `back` at the rows this rank sent it, [sum_{q'<q}
+ * send_rows[q'], ... + send_rows[q]), ready for ep_combine.  Arguments as
+ * for ep_dispatch_exchange.
+ */
+ep_status ep_combine_exchange(ep_nccl_comm comm, const void *expert_rows,
+                              const int32_t *recv_rows, const int32_t *send_rows,
+                              size_t row_bytes, void *back, ep_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char *ep_status_string(ep_status status);

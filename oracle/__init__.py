@@ -51,7 +51,7 @@ def lib() -> ctypes.CDLL:
         P, I, F, U8, U16 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                            ctypes.c_uint8, ctypes.c_uint16)
         _lib.orc_route.argtypes = [P, P, I, I, I, I, I, F, I, P, P, P]
-        _lib.orc_route.restype = None
+        _lib.orc_route.restype = I
         _lib.orc_layout.argtypes = [P, I, I, I, I, I, P, P, I, P, P, P, P, P, P, P, P]
         _lib.orc_layout.restype = I
         _lib.orc_layout_aligned.argtypes = [P, I, I, I, I, I, P, P, I, I, P, P, P, P, P, P, P, P]
@@ -154,6 +154,9 @@ def route(logits, bias, n_group: int, topk_group: int, topk: int,
     w = np.zeros((T, topk), dtype=np.float32)
     hard = np.zeros(T, dtype=np.uint8)
     L = lib()
+    if L.orc_route(None, None, 0, E, n_group, topk_group, topk, 1.0, 0, None, None, None):
+        raise ValueError(f"routing undefined for E={E}, n_group={n_group}, "
+                         f"topk_group={topk_group}, k={topk}")
 
     def part(t0, t1):
         L.orc_route(_ptr(lg[t0:t1]), _ptr(b), t1 - t0, E, n_group, topk_group, topk,

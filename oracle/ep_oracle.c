@@ -154,11 +154,20 @@ float orc_sigmoid(float x, int *hard)
  * logits [T,E], bias [E] or NULL (all zero), outputs topk_idx [T,k],
  * topk_w [T,k]; hard_tok [T] (optional) marks tokens holding a hard sigmoid.
  * Groups are n_group runs of E/n_group consecutive experts.
+ * Returns 0, or -1 (writing nothing) for a configuration the method does
+ * not define: E not a multiple of n_group, topk_group outside [1, n_group],
+ * k outside [1, (E/n_group) * topk_group], or, with more than one group,
+ * groups of a single expert (R3 scores a group by its TWO largest keys).
  */
-void orc_route(const float *logits, const float *bias, int T, int E,
-               int n_group, int topk_group, int k, float routed_scale,
-               int renorm, int32_t *topk_idx, float *topk_w, uint8_t *hard_tok)
+int orc_route(const float *logits, const float *bias, int T, int E,
+              int n_group, int topk_group, int k, float routed_scale,
+              int renorm, int32_t *topk_idx, float *topk_w, uint8_t *hard_tok)
 {
+    if (T < 0 || E < 1 || n_group < 1 || E % n_group != 0) return -1;
+    if (topk_group < 1 || topk_group > n_group) return -1;
+    if (k < 1 || k > (E / n_group) * topk_group) return -1;
+    if (n_group > 1 && E / n_group < 2) return -1;
+
     float *s = malloc(sizeof(float) * (size_t)E);
     float *key = malloc(sizeof(float) * (size_t)E);
     float *gscore = malloc(sizeof(float) * (size_t)n_group);
@@ -226,6 +235,7 @@ void orc_route(const float *logits, const float *bias, int T, int E,
         if (hard_tok) hard_tok[t] = (uint8_t)hard_any;
     }
     free(s); free(key); free(gscore); free(allowed); free(taken); free(gsel);
+    return 0;
 }
 
 /* ------------------------------------------------------------------ */

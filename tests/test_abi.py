@@ -20,6 +20,14 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", text)))
 
 
+# Every call below must fail its host checks.  They pass fake device
+# addresses, so this module only runs where no GPU is visible: a check that
+# went missing must never turn into a launch on real memory.
+pytestmark = pytest.mark.skipif(
+    __import__("torch").cuda.is_available(),
+    reason="host-check tests pass fake device pointers; run them where no GPU is visible")
+
+
 @pytest.fixture(scope="module")
 def lib():
     from combine_ep_route_02_b200 import build
@@ -154,3 +162,37 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         B.lib()
+
+
+def test_exchange_entry_points_reject_bad_arguments(lib):
+    """the NCCL exchange calls check their arguments before touching the
+    communicator (no GPU, no NCCL communicator needed)"""
+    import numpy as np
+    c = np.zeros(4, np.int32)
+    assert lib.ep_exchange_counts(None, FAKE, FAKE, 256, FAKE, FAKE, None) in (
+        B.EP_ERR_INVALID, B.EP_ERR_UNSUPPORTED)
+    assert lib.ep_exchange_counts(FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) in (
+        B.EP_ERR_INVALID, B.EP_ERR_UNSUPPORTED)
+    assert lib.ep_dispatch_exchange(None, FAKE, c.ctypes.data, c.ctypes.data, 16, FAKE,
+                                    None) == B.EP_ERR_INVALID
+    assert lib.ep_combine_exchange(None, FAKE, c.ctypes.data, c.ctypes.data, 16, FAKE,
+                                   None) == B.EP_ERR_INVALID
+
+
+def test_route_dispatch_rejects_invalid(lib):
+    cfg = B.RouteCfg(256, 8, 4, 8, 2.5, 1)
+    args = [FAKE, None, 16, cfg, 256, 8, None, None, 0, 1, FAKE, 7168, 1, 0, FAKE, FAKE,
+            FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, MIS, 0, None, None]
+    assert lib.ep_route_dispatch(*args) == B.EP_ERR_INVALID          # workspace misaligned
+    args[26] = FAKE
+    bad_h = list(args)
+    bad_h[11] = 7000                                                  # fp8 needs H % 128 == 0
+    assert lib.ep_route_dispatch(*bad_h) == B.EP_ERR_INVALID
+    bad_x = list(args)
+    bad_x[10] = MIS                                                   # x not 16-byte aligned
+    assert lib.ep_route_dispatch(*bad_x) == B.EP_ERR_INVALID
+
+
+def test_testing_knob_range(lib):
+    assert lib.ep_testing_set_wait_limit(1 << 33) == B.EP_ERR_INVALID
+    assert lib.ep_testing_set_wait_limit(-1) == B.EP_OK

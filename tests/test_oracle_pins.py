@@ -272,6 +272,43 @@ def test_route_single_group_is_plain_topk():
     assert np.array_equal(w[ok], np.take_along_axis(s.astype(np.float32), idx, 1)[ok])
 
 
+@pytest.mark.parametrize("E,G,Kg,k", [
+    (16, 16, 2, 2),   # groups of one expert: no second key to score a group by
+    (16, 3, 1, 2),    # E not a multiple of the group count
+    (16, 4, 5, 2),    # more groups kept than there are
+    (16, 4, 1, 5),    # more experts than the kept groups hold
+    (16, 1, 1, 0),
+])
+def test_route_rejects_undefined_configurations(E, G, Kg, k):
+    """the oracle refuses configurations the method leaves undefined (the
+    group score is the sum of a group's two largest keys, so a group needs
+    two experts) instead of reading past a group"""
+    logits = np.zeros((3, E), np.float32)
+    with pytest.raises(ValueError):
+        oracle.route(logits, None, G, Kg, k, 1.0, True)
+
+
+def test_route_two_expert_groups_brute_force():
+    """the smallest groups the method defines (two experts: the group score
+    is the sum of both keys) against exhaustive enumeration of group subsets"""
+    import itertools
+    rng = np.random.default_rng(17)
+    E, G, Kg, k = 8, 4, 2, 3
+    logits = rng.normal(0, 1, (64, E)).astype(np.float32)
+    idx, _, hard = oracle.route(logits, None, G, Kg, k, 1.0, False)
+    s = (1 / (1 + np.exp(-logits.astype(np.float64)))).astype(np.float32)
+    for t in range(64):
+        if hard[t]:
+            continue
+        gscore = [np.float32(s[t, 2 * g]) + np.float32(s[t, 2 * g + 1]) for g in range(G)]
+        best = max(itertools.combinations(range(G), Kg),
+                   key=lambda c: (sorted((gscore[g] for g in c), reverse=True),
+                                  [-g for g in c]))
+        allowed = [e for e in range(E) if e // 2 in best]
+        want = sorted(allowed, key=lambda e: (-s[t, e], e))[:k]
+        assert list(idx[t]) == want
+
+
 def test_route_invariants_v3_shape():
     cfg = CONFIGS["v3"].scaled(512)
     wl = Workload(cfg)

@@ -65,6 +65,9 @@ def test_noalloc_layout_matches_workspace_layout_twice():
     cases = [
         dict(T=16384, k=8, E=256, P=288, R=32, seed=1, replicas=True, bad=False),
         dict(T=1000, k=6, E=64, P=64, R=8, seed=2, replicas=False, bad=True),
+        # more than 64 tiles: the column-scan kernel rewrites the per-tile
+        # histograms in place, over what the previous call left there
+        dict(T=40000, k=8, E=256, P=256, R=8, seed=3, replicas=False, bad=False),
     ]
     for c in cases:
         T, k, E, P, R = c["T"], c["k"], c["E"], c["P"], c["R"]
