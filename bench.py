@@ -574,8 +574,14 @@ def main():
                     "timing": "CUDA events on the launching stream around each launch, "
                               "mean over the K eager steps",
                     # DRAM bytes need a profiler's counters, which this run does
-                    # not collect; the ncu captures are kept with the profiles
-                    "traffic": None}
+                    # not collect
+                    "traffic": None,
+                    "traffic_source": ("ncu capture of this kernel, one launch, in profiles/ "
+                                       "(" + ("route_dispatch_small_kernel_v3_decode.md"
+                                              if dom == "route_dispatch_small_kernel" else
+                                              "combine_kernel_v3_T2048.md"
+                                              if dom == "combine_kernel" else
+                                              "dispatch_fp8_tma_kernel_v3_T2048.md") + ")")}
         dc_ms = comb_ms + disp_ms
         extra = {
             "route_layout_us": None if fused else rl_ms * 1e3,
