@@ -12,7 +12,7 @@ import os
 
 import torch
 
-from .build import LIB
+from .build import LOAD_LIB as LIB
 
 _lib = None
 

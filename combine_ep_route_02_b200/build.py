@@ -18,6 +18,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libep_b200.so")
+# the library the binding loads: LIB, or another build of it named by
+# EP_B200_LIB (for example one installed elsewhere)
+LOAD_LIB = os.environ.get("EP_B200_LIB") or LIB
 HEADER = os.path.join(ROOT, "include", "ep.h")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

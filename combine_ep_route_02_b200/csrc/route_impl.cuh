@@ -91,11 +91,23 @@ EP_DEV double exp_table(double y, const double *tab)
     return e * __hiloint2double((1023 + (N >> 6)) << 20, 0);
 }
 
+// ---- the exact sigmoid rounded once to fp32 -----------------------------
+//
+// sigmoid_fast evaluates 1 / (1 + e^-x) in fp64 to within a few fp64 ulps and
+// rounds it to fp32; that is the correct rounding unless the fp64 value lies
+// within 64 fp64 ulps (about 2^-46, relative) of an fp32 rounding midpoint,
+// which sigmoid_fast reports in `near` (about one input in 2^22).  Those take
+// sigmoid_exact: the same quantity in double-double arithmetic (Dekker's
+// exact products and sums, error below 2^-95 relative) and a comparison with
+// the midpoint.  No fp32 input has a sigmoid closer than 2^-100 to a
+// midpoint, so the result is the exact value's rounding in every case.
+
 // s = fp32(1 / (1 + exp(-x))) from an fp64 evaluation accurate to a few
 // fp64 ulps (the reciprocal: a hardware estimate and two Newton steps).
-EP_DEV float sigmoid_f32(float x, const double *tab)
+EP_DEV float sigmoid_fast(float x, const double *tab, bool &near)
 {
     double y = -(double)x;
+    near = false;
     if (y > 700.0) return 0.0f;    // s < e^-700 rounds to +0 in fp32
     if (y < -700.0) y = -700.0;    // 1 + e^y rounds to 1 either way
     const double d = 1.0 + exp_table(y, tab);
@@ -103,7 +115,105 @@ EP_DEV float sigmoid_f32(float x, const double *tab)
     asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(z) : "d"(d));
     z = fma(z, fma(-d, z, 1.0), z);
     z = fma(z, fma(-d, z, 1.0), z);
-    return __double2float_rn(z);
+    const float f = __double2float_rn(z);
+    if (z >= 0x1p-126) {
+        // fp32 normal: rounding looks at the low 29 of the 52 fraction bits;
+        // 2^28 there is the midpoint
+        const int lo = (int)((uint32_t)__double2loint(z) & 0x1FFFFFFFu) - (1 << 28);
+        near = (unsigned)(lo + 64) <= 128u;
+    } else {
+        // fp32 subnormal (x below about -87): compare with the midpoint
+        const double fd = (double)f;
+        const double g = (double)__uint_as_float(z >= fd ? __float_as_uint(f) + 1u
+                                                          : __float_as_uint(f) - 1u);
+        near = fabs(z - 0.5 * (fd + g)) <= 0x1p-46 * z;
+    }
+    return f;
+}
+
+struct DD {
+    double hi, lo;
+};
+
+// a + b exactly, as hi + lo (Knuth)
+EP_DEV DD two_sum(double a, double b)
+{
+    const double s = __dadd_rn(a, b);
+    const double bb = __dsub_rn(s, a);
+    return {s, __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb))};
+}
+// a + b exactly for |a| >= |b| (Dekker)
+EP_DEV DD quick_two_sum(double a, double b)
+{
+    const double s = __dadd_rn(a, b);
+    return {s, __dsub_rn(b, __dsub_rn(s, a))};
+}
+EP_DEV DD dd_add(DD a, DD b)
+{
+    const DD s = two_sum(a.hi, b.hi);
+    const DD t = two_sum(a.lo, b.lo);
+    DD v = quick_two_sum(s.hi, __dadd_rn(s.lo, t.hi));
+    return quick_two_sum(v.hi, __dadd_rn(t.lo, v.lo));
+}
+EP_DEV DD dd_mul(DD a, DD b)
+{
+    const double p = __dmul_rn(a.hi, b.hi);
+    const double e = __fma_rn(a.hi, b.hi, -p);  // a.hi * b.hi - p, exact
+    const double t = __fma_rn(a.hi, b.lo, __fma_rn(a.lo, b.hi, e));
+    return quick_two_sum(p, t);
+}
+
+// The exact sigmoid rounded to fp32, for the inputs sigmoid_fast flags.
+// e^y with y = -x: y = N ln2 + r (ln2 in three parts, the first with 11
+// trailing zero bits so N times it is exact), e^r = (e^(r/256))^256 with
+// e^(r/256) - 1 from its Taylor series to degree 10 (remainder below 2^-104)
+// and eight squarings of 1 + p as p <- 2p + p^2; then 1 / (1 + e^y) by a
+// Newton step on the fp64 quotient, and the side of the fp32 midpoint.
+static __device__ __noinline__ float sigmoid_exact(float x)
+{
+    double y = -(double)x;
+    if (y > 700.0) return 0.0f;
+    if (y < -700.0) y = -700.0;
+    const double L1 = 0x1.62e42fefa3800p-1, L2 = 0x1.ef35793c76730p-45,
+                 L3 = 0x1.f97b57a079a19p-103;
+    const double N = rint(__dmul_rn(y, 0x1.71547652b82fep+0));  // y / ln2, to an integer
+    const double r_hi = __fma_rn(-N, L1, y);                    // exact
+    DD r = dd_add({r_hi, 0.0}, {__dmul_rn(-N, L2), __fma_rn(-N, L2, __dmul_rn(N, L2))});
+    r = dd_add(r, {__dmul_rn(-N, L3), 0.0});
+    r.hi = __dmul_rn(r.hi, 0x1p-8);  // r / 256, exact
+    r.lo = __dmul_rn(r.lo, 0x1p-8);
+    // 1/n! as two doubles each (hi = nearest double, lo = the remainder)
+    const DD c[11] = {{0.0, 0.0}, {1.0, 0.0}, {0.5, 0.0},
+                      {0x1.5555555555555p-3, 0x1.5555555555555p-57},
+                      {0x1.5555555555555p-5, 0x1.5555555555555p-59},
+                      {0x1.1111111111111p-7, 0x1.1111111111111p-63},
+                      {0x1.6c16c16c16c17p-10, -0x1.f49f49f49f49fp-65},
+                      {0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-73},
+                      {0x1.a01a01a01a01ap-16, 0x1.a01a01a01a01ap-76},
+                      {0x1.71de3a556c734p-19, -0x1.c154f8ddc6c00p-73},
+                      {0x1.27e4fb7789f5cp-22, 0x1.cbbc05b4fa99ap-76}};
+    DD p = c[10];
+    for (int n = 9; n >= 1; --n) p = dd_add(dd_mul(p, r), c[n]);
+    p = dd_mul(p, r);  // e^(r/256) - 1
+    for (int i = 0; i < 8; ++i) p = dd_add({__dmul_rn(p.hi, 2.0), __dmul_rn(p.lo, 2.0)}, dd_mul(p, p));
+    DD e = dd_add({1.0, 0.0}, p);  // e^r
+    const int n = (int)N;          // |N| <= 1010: scale by 2^N in two exact steps
+    const double s1 = __hiloint2double((1023 + n / 2) << 20, 0);
+    const double s2 = __hiloint2double((1023 + (n - n / 2)) << 20, 0);
+    e.hi = __dmul_rn(__dmul_rn(e.hi, s1), s2);
+    e.lo = __dmul_rn(__dmul_rn(e.lo, s1), s2);
+    const DD d = dd_add({1.0, 0.0}, e);
+    const double q = __ddiv_rn(1.0, d.hi);
+    // 1 - d q, exact for the hi part, then the lo part's share
+    const double res = __dsub_rn(__fma_rn(-d.hi, q, 1.0), __dmul_rn(d.lo, q));
+    const DD s = quick_two_sum(q, __dmul_rn(res, q));
+    const float lo32 = __double2float_rd(s.hi), hi32 = __double2float_ru(s.hi);
+    if (lo32 == hi32) return lo32;
+    const double mid = 0.5 * ((double)lo32 + (double)hi32);  // exact
+    const double t = __dadd_rn(__dsub_rn(s.hi, mid), s.lo);
+    if (t > 0.0) return hi32;
+    if (t < 0.0) return lo32;
+    return (__float_as_uint(lo32) & 1u) ? hi32 : lo32;  // a tie: to even (never met)
 }
 
 // winner of (key desc, index asc) over the warp; every lane gets it
@@ -161,18 +271,28 @@ EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restri
             for (int i = 0; i < EPL; ++i) x[i] = (e0 + i < E) ? __ldg(row + e0 + i) : 0.0f;
         }
 
-        // s = fp32(1 / (1 + exp(-x))) evaluated in fp64; key = fp32(s + b)
+        // s = the exact sigmoid rounded to fp32; key = fp32(s + b)
         float s[EPL];
         uint32_t key[EPL];
         uint32_t live = 0;  // bit i: expert e0+i exists and is still eligible
+        uint32_t near = 0;  // bit i: s[i] needs the exact evaluation
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            bool nr = false;
+            s[i] = (e0 + i < E) ? sigmoid_fast(x[i], tab, nr) : 0.0f;
+            near |= (uint32_t)nr << i;
+        }
+        if (__any_sync(FULL_MASK, near != 0)) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if ((near >> i) & 1u) s[i] = sigmoid_exact(x[i]);
+        }
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             if (e0 + i < E) {
-                s[i] = sigmoid_f32(x[i], tab);
                 key[i] = ordered(__fadd_rn(__fadd_rn(s[i], b[i]), 0.0f));
                 live |= 1u << i;
             } else {
-                s[i] = 0.0f;
                 key[i] = NONE;
             }
         }

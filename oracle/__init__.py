@@ -36,7 +36,7 @@ def build(force: bool = False) -> str:
         return _LIB
     os.makedirs(os.path.dirname(_LIB), exist_ok=True)
     tmp = _LIB + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lquadmath", "-lm"])
     os.replace(tmp, _LIB)
     return _LIB
 
@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
         _lib.orc_combine_backward.argtypes = [P, P, I, P, P, I, I, I, P, P]
         _lib.orc_combine_backward.restype = None
         S = ctypes.c_size_t
+        U32 = ctypes.c_uint32
+        _lib.orc_sigmoid_hard_scan.argtypes = [U32, U32, P, U32]
+        _lib.orc_sigmoid_hard_scan.restype = U32
         _lib.orc_e4m3_encode_array.argtypes = [P, S, P]
         _lib.orc_e4m3_encode_array.restype = None
         _lib.orc_bf16_encode_array.argtypes = [P, S, P]
@@ -134,6 +137,16 @@ def _run_ranges(fn, T: int, threads: int):
     with ThreadPoolExecutor(max_workers=len(ranges)) as ex:
         for f in [ex.submit(fn, *r) for r in ranges]:
             f.result()
+
+
+def sigmoid_hard_scan(first: int, count: int, cap: int = 1 << 16) -> np.ndarray:
+    """fp32 bit patterns in [first, first + count) whose sigmoid lies within
+    2^-47 of an fp32 rounding midpoint in fp64 (decided in quad precision)."""
+    out = np.zeros(cap, np.uint32)
+    n = int(lib().orc_sigmoid_hard_scan(first, count, out.ctypes.data, cap))
+    if n > cap:
+        raise RuntimeError("more hard inputs than the buffer holds")
+    return out[:n].copy()
 
 
 def sigmoid(x: float):

@@ -33,10 +33,12 @@
  *    rows, BF16 combine with fp32 accumulation.
  *
  * Readings where the pages are silent:
- *  R1 sigmoid: s = fp32_RN( 1 / (1 + exp(-x)) ) evaluated in fp64.  An
- *     element whose fp64 value lies within 2^-47 relative of an fp32 rounding
- *     midpoint is flagged "hard": another correct evaluation may round it to
- *     the other neighbour.
+ *  R1 sigmoid: s = the exact 1 / (1 + e^-x) rounded once to fp32 (nearest,
+ *     ties to even; a tie cannot occur: the value is irrational for x != 0).
+ *     It is evaluated in fp64 (error a few units of 2^-53); an element whose
+ *     fp64 value lies within 2^-47 (relative) of an fp32 rounding midpoint is
+ *     flagged "hard" and decided again in quad precision (113-bit
+ *     significand), far closer than any fp32 input comes to a midpoint.
  *  R2 the bias enters selection only: key = fp32_RN(s + b); weights use s.
  *  R3 group score = fp32_RN(k1 + k2), k1 >= k2 the two largest keys.
  *  R4 order: (key desc, index asc) for experts; (score desc, id asc) for
@@ -63,6 +65,7 @@
  *     and unused rows untouched.
  */
 #include <math.h>
+#include <quadmath.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -137,16 +140,58 @@ float orc_e4m3_decode(uint8_t c)
 /* routing                                                             */
 /* ------------------------------------------------------------------ */
 
-/* R1: fp64 sigmoid rounded once to fp32, with the hard-case flag. */
-float orc_sigmoid(float x, int *hard)
+/* fp64 sigmoid and whether it lies within 2^-47 (relative) of an fp32
+ * rounding midpoint (then fp64 cannot be trusted to round it). */
+static double sigmoid_fp64(float x, int *hard)
 {
     double v = 1.0 / (1.0 + exp(-(double)x));
     float f = (float)v;
     double fd = (double)f;
     float other = (v >= fd) ? nextafterf(f, INFINITY) : nextafterf(f, -INFINITY);
     double mid = 0.5 * (fd + (double)other); /* exact: adjacent floats */
-    if (hard) *hard = fabs(v - mid) <= ldexp(fabs(v), -47);
-    return f;
+    *hard = fabs(v - mid) <= ldexp(fabs(v), -47);
+    return v;
+}
+
+/* R1: the sigmoid correctly rounded to fp32, with the hard-case flag. */
+float orc_sigmoid(float x, int *hard)
+{
+    int h = 0;
+    double v = sigmoid_fp64(x, &h);
+    if (hard) *hard = h;
+    float f = (float)v;
+    if (!h) return f;
+    /* near a midpoint: the two fp32 neighbours, and the side of their
+     * midpoint on which the quad-precision value lies */
+    double fd = (double)f;
+    float other = (v >= fd) ? nextafterf(f, INFINITY) : nextafterf(f, -INFINITY);
+    float lo = fd < (double)other ? f : other;
+    float hi = fd < (double)other ? other : f;
+    __float128 q = 1.0Q / (1.0Q + expq(-(__float128)x));
+    __float128 m = ((__float128)lo + (__float128)hi) / 2; /* exact */
+    if (q > m) return hi;
+    if (q < m) return lo;
+    return (float_to_bits(lo) & 1u) ? hi : lo; /* a tie: to even (never met) */
+}
+
+/* Bit patterns b in [first, first + count) whose fp32 value's sigmoid is
+ * hard (see sigmoid_fp64); NaN patterns are skipped.  Writes up to cap of
+ * them to out and returns how many there are. */
+uint32_t orc_sigmoid_hard_scan(uint32_t first, uint32_t count, uint32_t *out, uint32_t cap)
+{
+    uint32_t n = 0;
+    for (uint32_t i = 0; i < count; ++i) {
+        uint32_t b = first + i;
+        float x = bits_to_float(b);
+        if (isnan(x)) continue;
+        int h = 0;
+        sigmoid_fp64(x, &h);
+        if (h) {
+            if (n < cap) out[n] = b;
+            ++n;
+        }
+    }
+    return n;
 }
 
 /*
