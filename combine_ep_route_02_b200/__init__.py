@@ -10,6 +10,7 @@ call does, and raises if it has not been built.
 from ._binding import (  # noqa: F401
     EP_DEV_BAD_EXPERT,
     EP_DEV_BAD_REPLICA,
+    EP_DEV_OVERFLOW,
     EP_DEV_TIMEOUT,
     EP_ERR_CUDA,
     EP_ERR_DEVICE,
@@ -35,3 +36,4 @@ from ._binding import (  # noqa: F401
 from .exchange import (ExchangePlan, combine_exchange, dispatch_exchange,  # noqa: F401
                        exchange_plan)
 from .path import EpHostPipeline, EpMicroBatchPipeline, EpPath  # noqa: F401
+from .peer import EpPeerRanks  # noqa: F401

@@ -30,7 +30,9 @@ EXPORTS = ("ep_workspace_size", "ep_route", "ep_dispatch_layout", "ep_dispatch",
            "ep_combine", "ep_status_string", "ep_dispatch_layout_noalloc", "ep_route_layout",
            "ep_dispatch_backward", "ep_combine_backward", "ep_silu_mul", "ep_route_dispatch",
            "ep_testing_set_wait_limit", "ep_exchange_counts", "ep_dispatch_exchange",
-           "ep_combine_exchange")
+           "ep_combine_exchange", "ep_peer_counts", "ep_peer_dispatch", "ep_peer_wait_dispatch",
+           "ep_peer_experts_ready", "ep_peer_combine")
+EP_DEV_OVERFLOW = 8
 
 
 class EpError(RuntimeError):
@@ -44,6 +46,25 @@ class RouteCfg(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int), ("n_group", ctypes.c_int),
                 ("topk_group", ctypes.c_int), ("topk", ctypes.c_int),
                 ("routed_scale", ctypes.c_float), ("renorm", ctypes.c_int)]
+
+
+class PeerGroup(ctypes.Structure):
+    """ep_peer_group: the rank-indexed tables are device addresses of arrays
+    of W device pointers."""
+    _fields_ = [("world", ctypes.c_int), ("rank0", ctypes.c_int), ("n_local", ctypes.c_int),
+                ("P", ctypes.c_int), ("row_align", ctypes.c_int), ("cap", ctypes.c_int),
+                ("recv_x", ctypes.c_void_p), ("recv_scale", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("board", ctypes.c_void_p), ("flags", ctypes.c_void_p)]
+
+
+class PeerRank(ctypes.Structure):
+    """ep_peer_rank: one local rank's own arrays (device addresses)."""
+    _fields_ = [("x", ctypes.c_void_p), ("cnt_expert", ctypes.c_void_p),
+                ("expert_off", ctypes.c_void_p), ("slot", ctypes.c_void_p),
+                ("topk_w", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("dest_off", ctypes.c_void_p), ("recv_cnt", ctypes.c_void_p),
+                ("recv_rows", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
+                ("T", ctypes.c_int), ("reserved", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -90,6 +111,17 @@ def lib() -> ctypes.CDLL:
         L.ep_dispatch_exchange.restype = I
         L.ep_combine_exchange.argtypes = [P, P, P, P, Z, P, P]
         L.ep_combine_exchange.restype = I
+        G, RP = PeerGroup, ctypes.c_void_p
+        L.ep_peer_counts.argtypes = [G, RP, P]
+        L.ep_peer_counts.restype = I
+        L.ep_peer_dispatch.argtypes = [G, RP, I, I, I, P]
+        L.ep_peer_dispatch.restype = I
+        L.ep_peer_wait_dispatch.argtypes = [G, RP, P]
+        L.ep_peer_wait_dispatch.restype = I
+        L.ep_peer_experts_ready.argtypes = [G, P]
+        L.ep_peer_experts_ready.restype = I
+        L.ep_peer_combine.argtypes = [G, RP, I, I, I, P]
+        L.ep_peer_combine.restype = I
         L.ep_status_string.argtypes = [I]
         L.ep_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -223,6 +255,30 @@ def ep_combine_exchange(comm: int, expert_rows, recv_rows, send_rows, row_bytes:
     _check("ep_combine_exchange", lib().ep_combine_exchange(
         comm, _ptr(expert_rows), r.ctypes.data, s.ctypes.data, row_bytes, _ptr(back),
         _stream(stream)))
+
+
+def ep_peer_counts(group: PeerGroup, ranks_dev, stream=None):
+    """ranks_dev: device buffer holding n_local PeerRank structs."""
+    _check("ep_peer_counts", lib().ep_peer_counts(group, _ptr(ranks_dev), _stream(stream)))
+
+
+def ep_peer_dispatch(group: PeerGroup, ranks_dev, H, k, max_T, stream=None):
+    _check("ep_peer_dispatch", lib().ep_peer_dispatch(group, _ptr(ranks_dev), H, k, max_T,
+                                                      _stream(stream)))
+
+
+def ep_peer_wait_dispatch(group: PeerGroup, ranks_dev, stream=None):
+    _check("ep_peer_wait_dispatch", lib().ep_peer_wait_dispatch(group, _ptr(ranks_dev),
+                                                                _stream(stream)))
+
+
+def ep_peer_experts_ready(group: PeerGroup, stream=None):
+    _check("ep_peer_experts_ready", lib().ep_peer_experts_ready(group, _stream(stream)))
+
+
+def ep_peer_combine(group: PeerGroup, ranks_dev, H, k, max_T, stream=None):
+    _check("ep_peer_combine", lib().ep_peer_combine(group, _ptr(ranks_dev), H, k, max_T,
+                                                    _stream(stream)))
 
 
 def ep_dispatch_backward(grad_recv, slot, T, H, k, grad_x, num_sms=0, dev_status=None,

@@ -72,9 +72,11 @@ typedef enum {
 /* Bits reported through a caller's *dev_status word. */
 #define EP_DEV_BAD_EXPERT 1  /* layout: a topk_idx entry outside [0, E) */
 #define EP_DEV_BAD_REPLICA 2 /* layout: n_rep[e] outside [1, max_rep] or phys id outside [0, P) */
-#define EP_DEV_TIMEOUT 4     /* dispatch / route_dispatch: a bounded wait (for an
-                                asynchronous copy, or for the other blocks of the grid)
-                                gave up; that call's output is incomplete */
+#define EP_DEV_TIMEOUT 4     /* dispatch / route_dispatch / peer calls: a bounded wait (for
+                                an asynchronous copy, for the other blocks of the grid, or
+                                for another rank) gave up; that call's output is incomplete */
+#define EP_DEV_OVERFLOW 8    /* peer dispatch: a destination row beyond the receive
+                                buffers' capacity (the pair was skipped) */
 
 /* Same object as cudaStream_t; no CUDA header is needed to use this API. */
 typedef struct CUstream_st *ep_stream_t;
@@ -427,6 +429,92 @@ ep_status ep_dispatch_exchange(ep_nccl_comm comm, const void *rows, const int32_
 ep_status ep_combine_exchange(ep_nccl_comm comm, const void *expert_rows,
                               const int32_t *recv_rows, const int32_t *send_rows,
                               size_t row_bytes, void *back, ep_stream_t stream);
+
+/*
+ * Expert parallelism over peer memory (NVLink / NVSwitch): the dispatch and
+ * combine all-to-alls of the Perplexity blog (section "Expert Parallelism")
+ * as direct stores into, and loads from, the other ranks' buffers, with no
+ * collective library: the FP8 dispatch quantises each token once and stores
+ * its k rows straight into the receive buffers of the ranks that own the
+ * experts, and the combine gathers the expert outputs straight from them.
+ *
+ * W ranks; rank q owns physical experts [q*P/W, (q+1)*P/W).  A process
+ * serves ranks rank0 .. rank0 + n_local - 1 on its GPU: one rank per GPU
+ * across processes, or several ranks in one process (then the calls below
+ * cover all of them in one launch, and n_local must not exceed the SM count,
+ * since those blocks wait for one another).  Each rank's tokens are laid
+ * out first with ep_dispatch_layout (or ep_route_layout) with R = W and
+ * row_align 1; the peer calls read cnt_expert, expert_off, slot and topk_w.
+ *
+ * Rank q receives, for each of its experts e in order, the rows of source
+ * rank 0, then source 1, ..., each source's rows in its own (t, j) order;
+ * every expert's rows start on a multiple of row_align (the GEMM layout).
+ *
+ * Step protocol (every rank makes the same calls in the same order):
+ *   ep_peer_counts        all-gather of the per-expert counts through the
+ *                         boards; each rank computes where its rows go
+ *   ep_peer_dispatch      quantise + store rows to their owners, then tell
+ *                         every rank this source is complete
+ *   ep_peer_wait_dispatch a rank waits for all sources (before its experts)
+ *   (the rank's experts turn recv_x into y)
+ *   ep_peer_experts_ready a rank publishes that its y is complete
+ *   ep_peer_combine       weighted sum of each token's k rows read from the
+ *                         ranks that hold them (waits for their publication)
+ * Every wait is bounded: a wait that gives up ORs EP_DEV_TIMEOUT into the
+ * rank's dev_status and leaves that step's output incomplete.
+ *
+ * Buffers (all allocated by the caller).  Rank-indexed tables are DEVICE
+ * arrays of W device pointers, entry q being rank q's buffer as this process
+ * addresses it (its own allocation for a local rank; on one node, a CUDA IPC
+ * mapping of a peer's allocation).  Rank q's buffers: recv_x e4m3 [cap, H],
+ * recv_scale fp32 [cap, H/128], y bf16 [cap, H], board int32 [W, P], flags
+ * int32 [8] (zeroed once when allocated, then left to the library: they
+ * count the steps).  cap must hold every row rank q can receive: the sum of
+ * all sources' T*k plus (P/W)*(row_align-1); rows beyond cap are skipped and
+ * reported as EP_DEV_OVERFLOW.  No TMA and no multicast is used.
+ */
+typedef struct {
+    int world;                /* W */
+    int rank0;                /* first rank served by this process */
+    int n_local;              /* ranks served by this process */
+    int P;                    /* physical experts, a multiple of W */
+    int row_align;            /* expert row tile at the destinations (1..1024) */
+    int cap;                  /* rows of every rank's receive buffers */
+    void *const *recv_x;      /* [W] -> e4m3 [cap, H] */
+    float *const *recv_scale; /* [W] -> fp32 [cap, H/128] */
+    const void *const *y;     /* [W] -> bf16 [cap, H], expert outputs in receive order */
+    int32_t *const *board;    /* [W] -> int32 [W, P] */
+    int32_t *const *flags;    /* [W] -> int32 [8] */
+} ep_peer_group;
+
+/* One local rank's own arrays (a device array of n_local of these, in rank
+ * order, is passed to the calls). */
+typedef struct {
+    const void *x;              /* bf16 [T, H] tokens */
+    const int32_t *cnt_expert;  /* [P]   from its layout (R = W) */
+    const int32_t *expert_off;  /* [P+1] */
+    const int32_t *slot;        /* [T, k] */
+    const float *topk_w;        /* [T, k] */
+    void *out;                  /* bf16 [T, H] (out): combine */
+    int32_t *dest_off;          /* [P] (out): first row, at expert p's rank, of this
+                                   rank's rows for expert p (-1 after a timeout) */
+    int32_t *recv_cnt;          /* [P/W, W] (out): pairs from each source for each of
+                                   this rank's experts (for its grouped GEMM) */
+    int32_t *recv_rows;         /* [1] (out): rows this rank receives, padding included */
+    int32_t *dev_status;        /* [1] or NULL: EP_DEV_* bits are ORed in */
+    int T;                      /* tokens of this rank */
+    int reserved;
+} ep_peer_rank;
+
+ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, ep_stream_t stream);
+/* H % 128 == 0; k <= 32; max_T: the largest T of the local ranks (sizes the grid). */
+ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, int k,
+                           int max_T, ep_stream_t stream);
+ep_status ep_peer_wait_dispatch(ep_peer_group g, const ep_peer_rank *ranks, ep_stream_t stream);
+ep_status ep_peer_experts_ready(ep_peer_group g, ep_stream_t stream);
+/* out[t] = bf16(sum_j fp32(w[t,j] * y_q[row])) in j order, as ep_combine; H % 8 == 0. */
+ep_status ep_peer_combine(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int max_T,
+                          ep_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char *ep_status_string(ep_status status);
