@@ -288,6 +288,9 @@ def main():
                     help="skip timing the GEMM layout (padded rows) and the expert activation")
     ap.add_argument("--row-align", type=int, default=128,
                     help="row tile of the GEMM layout timed after the step")
+    ap.add_argument("--peer-ranks", type=int, default=8,
+                    help="also time the peer-memory expert-parallel dispatch and combine with "
+                         "this many ranks on this GPU (0 = skip)")
     ap.add_argument("--dry-run", action="store_true",
                     help="no GPU: check the multi-rank launch, the max-over-ranks timing and "
                          "the output line with gloo ranks running the CPU oracle")
@@ -597,6 +600,64 @@ def main():
             "step_us": tot_ms / K * 1e3,
         }
 
+    # expert parallelism over peer memory, every rank on this GPU: the
+    # workload's tokens split over `peer_ranks` ranks (R = that many), each
+    # with its own buffers addressed through the rank tables a multi-GPU
+    # group uses; events around the fused quantise + store dispatch and the
+    # gathering combine (stores and loads stay in this GPU's HBM here, where
+    # a multi-GPU group crosses NVLink)
+    peer = None
+    if args.peer_ranks > 1 and cfg.fp8 and cfg.T % args.peer_ranks == 0 and world == 1:
+        import dataclasses
+
+        from combine_ep_route_02_b200 import EpPeerRanks
+        Wp = args.peer_ranks
+        pcfg = dataclasses.replace(cfg.scaled(cfg.T // Wp), R=Wp)
+        pwls = [Workload(pcfg, seed=1000 + r) for r in range(Wp)]
+        ppaths = [EpPath(pcfg.T, pcfg.H, pcfg.E, pcfg.n_group, pcfg.topk_group, pcfg.topk,
+                         pcfg.routed_scale, pcfg.renorm, Wp, True, phys_of=w.phys_of,
+                         n_rep=w.n_rep) for w in pwls]
+        for pp_, w in zip(ppaths, pwls):
+            pp_.route_layout(w.logits.cuda(), w.bias.cuda())
+        grp = EpPeerRanks.local(ppaths, pcfg.H)
+        pxs = [w.x.cuda() for w in pwls]
+        pouts = [torch.empty((pcfg.T, pcfg.H), dtype=torch.bfloat16, device="cuda")
+                 for _ in range(Wp)]
+        grp.set_inputs(pxs, pouts)
+        for i, yq in enumerate(grp.y):
+            yq.copy_(device_normal_bf16(grp.cap, pcfg.H, seed=2000 + i))
+        Kp = max(3, min(K, 50))
+        q0, q1, q2, q3 = (events(Kp) for _ in range(4))
+        for i in range(args.warmup + Kp):
+            j = i - args.warmup
+            grp.counts()
+            if j >= 0:
+                q0[j].record(stream)
+            grp.dispatch()
+            if j >= 0:
+                q1[j].record(stream)
+            grp.wait_dispatch()
+            grp.experts_ready()
+            if j >= 0:
+                q2[j].record(stream)
+            grp.combine()
+            if j >= 0:
+                q3[j].record(stream)
+        torch.cuda.synchronize()
+        if any(grp.check_status()):
+            raise RuntimeError(f"peer step status {grp.check_status()}")
+        pd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(q0, q1))
+        pc_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(q2, q3))
+        pab = algorithmic_bytes(pcfg)
+        pd_bytes, pc_bytes = pab["dispatch"] * Wp, pab["combine"] * Wp
+        peer = {"ranks": Wp, "tokens_per_rank": pcfg.T,
+                "dispatch_us": pd_ms * 1e3, "dispatch_gbs": pd_bytes / (pd_ms * 1e-3) / 1e9,
+                "combine_us": pc_ms * 1e3, "combine_gbs": pc_bytes / (pc_ms * 1e-3) / 1e9,
+                "dispatch_combine_tokens_per_s": cfg.T / ((pd_ms + pc_ms) * 1e-3),
+                "note": "all ranks on one GPU (one launch covers them); algorithmic bytes "
+                        "as for dispatch and combine, summed over the ranks"}
+        del grp, ppaths, pxs, pouts
+
     # end to end through the public API: every step uploads its inputs from
     # pinned host memory and downloads its result; EpHostPipeline overlaps
     # those copies with the neighbouring steps' compute
@@ -681,6 +742,7 @@ def main():
             "cpu_baseline": cpu,
             "backward": backward,
             "gemm_layout": gemm,
+            "peer_ep": peer,
             "clocks": sampler.summary(t_wall0, t_wall1),
             "wall_s_timed": t_wall1 - t_wall0,
             **extra,

@@ -23,7 +23,9 @@
 //
 // The grid has at most one block per SM (grid <= SM count), so every block
 // is resident; the wait still gives up after a bounded number of polls and
-// reports EP_DEV_TIMEOUT instead of hanging.
+// reports EP_DEV_TIMEOUT instead of hanging.  The counters live in the
+// caller's workspace: zero before its first use, and the last block to leave
+// clears them again (after a timeout too), so no call needs a memset.
 #include "layout_impl.cuh"
 #include "quant.cuh"
 #include "route_impl.cuh"
@@ -43,7 +45,8 @@ struct DecodeArgs {
     float *recv_scale;   // [n_rows, H/128] when fp8
     int tpb;             // tokens per block
     int scale_bulk;      // scale rows go out by bulk stores (16-byte rows, aligned)
-    int *ctrl;           // workspace: [0] arrivals, [1] departures, [2] status bits
+    int *ctrl;           // workspace: [0] arrivals, [1] departures, [2] status bits;
+                         // zero before the first call, left zero by every call
     uint32_t wait_limit; // polls of each bounded wait
 };
 
@@ -342,8 +345,13 @@ route_dispatch_small_kernel(RouteArgs r, LayoutArgs a, DecodeArgs d, int vec4)
         if (status) atomicOr(&d.ctrl[2], status);
         __threadfence();
         if (atomicAdd(&d.ctrl[1], 1) == NB - 1) {
+            // every block has left: publish the status and clear the words
+            // for the next call (it starts after this grid has finished)
             __threadfence();
             if (a.dev_status != nullptr) *a.dev_status = (int)ld_acquire(&d.ctrl[2]);
+            d.ctrl[0] = 0;
+            d.ctrl[1] = 0;
+            d.ctrl[2] = 0;
         }
     }
 }
@@ -382,9 +390,6 @@ cudaError_t launch_route_dispatch_small(const RouteArgs &r, LayoutArgs a, const 
     const int T = r.T;
     const int tpb = decode_tpb(T, sms);
     const int nb = (T + tpb - 1) / tpb;
-    // arrival, departure and status words start at zero on every call
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, 4 * sizeof(int), s);
-    if (e != cudaSuccess) return e;
     const int S = H / 128;
     DecodeArgs d{static_cast<const uint16_t *>(x), H, fp8, n_rows,
                  static_cast<uint8_t *>(recv_x), recv_scale, tpb,

@@ -275,8 +275,10 @@ ep_status ep_route_dispatch(const float *logits, const float *bias, int T, ep_ro
         const LayoutArgs a = layout_args(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep,
                                          row_align, cnt_expert, expert_off, rows_rank, rank_off,
                                          tok_rank, in_rank, slot, src, workspace, dev_status);
+        // the fused kernel's counters: 64 bytes into the workspace tail (the
+        // first bytes of the tail are the small-batch layout's counter)
         int *ctrl = reinterpret_cast<int *>(static_cast<char *>(workspace) +
-                                            layout_workspace_core(T, k, P, R));
+                                            layout_workspace_core(T, k, P, R) + 64);
         return from_cuda(launch_route_dispatch_small(r, a, x_bf16, H, fp8 != 0, n_rows, recv_x,
                                                      recv_scale, sms, ctrl, wait_limit(), s));
     }

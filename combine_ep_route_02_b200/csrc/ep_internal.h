@@ -140,7 +140,8 @@ struct ActivationArgs {
 
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 // workspace bytes: tile_cnt, tile_tok, tile_bad, each 256-byte aligned, then
-// 256 bytes holding the fused small-batch kernel's completion counter
+// 256 bytes: the small-batch layout kernel's completion counter at +0 and the
+// route + dispatch kernel's counters at +64
 inline size_t layout_workspace_core(int T, int k, int P, int R)
 {
     const size_t NT = (size_t)layout_tiles(T > 0 ? T : 1, k, P);
@@ -183,7 +184,8 @@ bool small_route_layout_ok(int T, int k, int P);
 cudaError_t launch_route_layout_small(const RouteArgs &r, LayoutArgs a, int *done,
                                       cudaStream_t s);
 // Fused routing + layout + dispatch for small batches (one kernel; see
-// decode.cu).  ctrl: 4 ints of workspace (zeroed by the launch).
+// decode.cu).  ctrl: 4 ints of workspace, zero before the first launch and
+// left zero by every launch.
 bool small_route_dispatch_ok(int T, int k, int P, int H, int fp8, int sms);
 cudaError_t launch_route_dispatch_small(const RouteArgs &r, LayoutArgs a, const void *x, int H,
                                         int fp8, int n_rows, void *recv_x, float *recv_scale,

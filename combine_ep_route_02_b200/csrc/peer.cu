@@ -78,10 +78,30 @@ EP_DEV void report(const ep_peer_rank &r, int bits)
     if (r.dev_status != nullptr) atomicOr(r.dev_status, bits);
 }
 
+// destination rank and row of pair (t, j) of a local rank, from its local
+// receive row (the layout's slot): expert p holds local rows
+// [expert_off[p], expert_off[p+1]); -1 rank when the pair is invalid
+EP_DEV void pair_dest(const int *eoff, const int *doff, int P, int epr, int s_loc, int &q,
+                      int &row)
+{
+    q = -1;
+    row = 0;
+    if (s_loc < 0 || s_loc >= eoff[P]) return;
+    int lo = 0, hi = P;  // eoff[lo] <= s_loc < eoff[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (eoff[mid] <= s_loc) lo = mid;
+        else hi = mid;
+    }
+    if (doff[lo] < 0) return;  // the counts step gave up
+    q = lo / epr;
+    row = doff[lo] + (s_loc - eoff[lo]);
+}
+
 // 1. all-gather of the per-expert counts, then this rank's destination
 //    offsets and receive counts.  One block per local rank.
 __global__ void __launch_bounds__(PEER_THREADS)
-peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
+peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t limit)
 {
     extern __shared__ int sm[];
     __shared__ int warp_tot[PEER_THREADS / 32 + 1];
@@ -89,8 +109,10 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
     const int W = g.world, P = g.P, epr = P / W, A = g.row_align;
     const int l = blockIdx.x, me = g.rank0 + l, tid = threadIdx.x;
     const ep_peer_rank &r = ranks[l];
-    int *tot = sm;           // [P] padded totals over all sources, then their scan
-    int *pre = sm + P;       // [P] rows of sources before this one
+    int *tot = sm;            // [P] padded totals over all sources, then their scan
+    int *pre = sm + P;        // [P] rows of sources before this one
+    int *eoff = sm + 2 * P;   // [P + 1] this rank's local expert offsets
+    int *doff = eoff + P + 1; // [P] destination offsets
     int32_t *my_flags = g.flags[me];
 
     pdl_launch_dependents();
@@ -113,6 +135,7 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
     if (!ok_sh) {
         // no destination rows: the dispatch and combine skip every pair
         for (int p = tid; p < P; p += PEER_THREADS) r.dest_off[p] = -1;
+        for (int i = tid; i < r.T * k; i += PEER_THREADS) r.pair_rank[i] = -1;
         if (tid == 0) {
             *r.recv_rows = 0;
             report(r, PEER_TIMEOUT);
@@ -139,94 +162,73 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
     const int total = layout_impl::block_exclusive_scan<PEER_THREADS>(tot, P, warp_tot);
     for (int p = tid; p < P; p += PEER_THREADS) {
         const int q = p / epr;
-        r.dest_off[p] = tot[p] - tot[q * epr] + pre[p];
+        doff[p] = tot[p] - tot[q * epr] + pre[p];
+        r.dest_off[p] = doff[p];
     }
+    for (int p = tid; p <= P; p += PEER_THREADS) eoff[p] = r.expert_off[p];
     if (tid == 0) {
         const int end = me + 1 < W ? tot[(me + 1) * epr] : total;
         *r.recv_rows = end - tot[me * epr];
     }
-}
-
-// destination rank and row of pair (t, j) of a local rank, from its local
-// receive row (the layout's slot): expert p holds local rows
-// [expert_off[p], expert_off[p+1]); -1 rank when the pair is invalid
-EP_DEV void pair_dest(const int *eoff, const int *doff, int P, int epr, int s_loc, int &q,
-                      int &row)
-{
-    q = -1;
-    row = 0;
-    if (s_loc < 0 || s_loc >= eoff[P]) return;
-    int lo = 0, hi = P;  // eoff[lo] <= s_loc < eoff[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (eoff[mid] <= s_loc) lo = mid;
-        else hi = mid;
+    __syncthreads();
+    // every pair's destination rank and row, for the dispatch and combine
+    int overflow = 0;
+    for (int i = tid; i < r.T * k; i += PEER_THREADS) {
+        int q, row;
+        pair_dest(eoff, doff, P, epr, r.slot[i], q, row);
+        if (q >= 0 && row >= g.cap) {
+            overflow = PEER_OVERFLOW;
+            q = -1;
+        }
+        r.pair_rank[i] = q;
+        r.pair_row[i] = row;
     }
-    if (doff[lo] < 0) return;  // the counts step gave up
-    q = lo / epr;
-    row = doff[lo] + (s_loc - eoff[lo]);
+    if (overflow) report(r, overflow);
 }
 
 // 2. dispatch: each token's row quantised once (1x128 e4m3) and stored k
 //    times into the owning ranks' receive buffers; the last block of a rank
 //    tells every destination that this source's rows are complete.
-//    Grid: n_local x bpr blocks.
+//    Grid: n_local x bpr blocks; within a rank, a thread owns a 16-element
+//    chunk of a row at a time (the flat walk of the local dispatch), and the
+//    8 lanes of a 128-element block reduce its amax together.
 __global__ void __launch_bounds__(PEER_THREADS)
 peer_dispatch_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int bpr)
 {
-    extern __shared__ int sm[];
-    __shared__ int dq[MAX_TOPK], drow[MAX_TOPK];
     __shared__ int last_sh;
-    const int W = g.world, P = g.P, epr = P / W;
+    const int W = g.world;
     const int l = blockIdx.x / bpr, part = blockIdx.x % bpr, me = g.rank0 + l;
     const int tid = threadIdx.x;
     const ep_peer_rank &r = ranks[l];
-    int *eoff = sm;          // [P + 1]
-    int *doff = sm + P + 1;  // [P]
     pdl_launch_dependents();
     pdl_wait();
-    for (int p = tid; p <= P; p += PEER_THREADS) eoff[p] = r.expert_off[p];
-    for (int p = tid; p < P; p += PEER_THREADS) doff[p] = r.dest_off[p];
-    __syncthreads();
-    const int S = H >> 7, cpr = H >> 4;
+    const int S = H >> 7, cpr = H >> 4;  // cpr is a multiple of 8
     const uint16_t *x = static_cast<const uint16_t *>(r.x);
-    int overflow = 0;
-    for (int t = part; t < r.T; t += bpr) {  // block-uniform
-        if (tid < k) {
-            int q, row;
-            pair_dest(eoff, doff, P, epr, r.slot[(size_t)t * k + tid], q, row);
-            if (q >= 0 && row >= g.cap) {
-                overflow = PEER_OVERFLOW;
-                q = -1;
-            }
-            dq[tid] = q;
-            drow[tid] = row;
+    const long long total = (long long)r.T * cpr;
+    const long long stride = (long long)bpr * PEER_THREADS;
+    ChunkWalk it((long long)part * PEER_THREADS + tid, stride, cpr);
+    // block-uniform bound: every lane reaches the shuffles; total and the
+    // stride are multiples of 8, so a lane octet is all active or all idle
+    for (long long base = (long long)part * PEER_THREADS; base < total; base += stride, it.next()) {
+        const bool active = it.t < r.T;
+        const int t = it.t, c = it.c;
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+        if (active) {
+            lo = ld_stream(x + (size_t)t * H + (size_t)c * 16);
+            hi = ld_stream(x + (size_t)t * H + (size_t)c * 16 + 8);
         }
-        __syncthreads();
-        // chunk c0 + tid: the 8 lanes of a 128-element block are all active
-        // or all idle (cpr is a multiple of 8, the stride of 256 too)
-        for (int c0 = 0; c0 < cpr; c0 += PEER_THREADS) {
-            const int c = c0 + tid;
-            const bool act = c < cpr;
-            uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-            if (act) {
-                lo = ld_stream(x + (size_t)t * H + (size_t)c * 16);
-                hi = ld_stream(x + (size_t)t * H + (size_t)c * 16 + 8);
+        float scale;
+        const uint4 qv = quant::quant_chunk(lo, hi, scale);
+        if (active)
+            for (int j = 0; j < k; ++j) {
+                const int q = __ldg(r.pair_rank + (size_t)t * k + j);
+                if (q < 0) continue;
+                const size_t row = (size_t)__ldg(r.pair_row + (size_t)t * k + j);
+                uint8_t *dst = static_cast<uint8_t *>(g.recv_x[q]) + row * H;
+                *reinterpret_cast<uint4 *>(dst + (size_t)c * 16) = qv;
+                if ((c & 7) == 0) g.recv_scale[q][row * S + (c >> 3)] = scale;
             }
-            float scale;
-            const uint4 qv = quant::quant_chunk(lo, hi, scale);
-            if (act)
-                for (int j = 0; j < k; ++j) {
-                    const int q = dq[j];
-                    if (q < 0) continue;
-                    uint8_t *dst = static_cast<uint8_t *>(g.recv_x[q]) + (size_t)drow[j] * H;
-                    *reinterpret_cast<uint4 *>(dst + (size_t)c * 16) = qv;
-                    if ((c & 7) == 0) g.recv_scale[q][(size_t)drow[j] * S + (c >> 3)] = scale;
-                }
-        }
-        __syncthreads();
     }
-    if (overflow && tid < k) report(r, overflow);
     // this block's rows are visible everywhere before it counts itself done
     __threadfence_system();
     __syncthreads();
@@ -273,21 +275,17 @@ __global__ void peer_ready_kernel(ep_peer_group g)
 // 5. combine: once every rank holding this rank's pairs has its outputs
 //    ready, each token's k rows are read from those ranks and summed in j
 //    order with the weights, in fp32, rounded once to bf16 (as ep_combine).
-//    Grid: n_local x bpr blocks; a thread owns 8 elements of a row.
+//    Grid: n_local x bpr blocks; a thread owns an 8-element chunk of an
+//    output row and issues up to 8 row loads before it accumulates.
 __global__ void __launch_bounds__(PEER_THREADS)
 peer_combine_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int bpr,
                     uint32_t limit)
 {
-    extern __shared__ int sm[];
-    __shared__ int dq[MAX_TOPK], drow[MAX_TOPK];
-    __shared__ float dw[MAX_TOPK];
     __shared__ int ok_sh;
-    const int W = g.world, P = g.P, epr = P / W;
+    const int W = g.world;
     const int l = blockIdx.x / bpr, part = blockIdx.x % bpr, me = g.rank0 + l;
     const int tid = threadIdx.x;
     const ep_peer_rank &r = ranks[l];
-    int *eoff = sm;
-    int *doff = sm + P + 1;
     pdl_launch_dependents();
     pdl_wait();
     if (tid == 0) {
@@ -297,47 +295,53 @@ peer_combine_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, in
         ok_sh = ok;
         if (!ok) report(r, PEER_TIMEOUT);
     }
-    for (int p = tid; p <= P; p += PEER_THREADS) eoff[p] = r.expert_off[p];
-    for (int p = tid; p < P; p += PEER_THREADS) doff[p] = r.dest_off[p];
     __syncthreads();
     if (!ok_sh) return;
+    constexpr int BATCH = 8;
     const int cpr = H >> 3;
     uint16_t *out = static_cast<uint16_t *>(r.out);
-    for (int t = part; t < r.T; t += bpr) {
-        if (tid < k) {
-            int q, row;
-            pair_dest(eoff, doff, P, epr, r.slot[(size_t)t * k + tid], q, row);
-            if (q >= 0 && row >= g.cap) q = -1;
-            dq[tid] = q;
-            drow[tid] = row;
-            dw[tid] = r.topk_w[(size_t)t * k + tid];
-        }
-        __syncthreads();
-        for (int c = tid; c < cpr; c += PEER_THREADS) {
-            float acc[8];
+    const long long total = (long long)r.T * cpr;
+    const long long g0 = (long long)part * PEER_THREADS + tid;
+    if (g0 >= total) return;
+    for (ChunkWalk it(g0, (long long)bpr * PEER_THREADS, cpr); it.t < r.T; it.next()) {
+        const int t = it.t, c = it.c;
+        float acc[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-            for (int j = 0; j < k; ++j) {
-                const int q = dq[j];
-                if (q < 0) continue;
-                const uint16_t *yq = static_cast<const uint16_t *>(g.y[q]);
-                const uint4 v = ld_stream(yq + (size_t)drow[j] * H + (size_t)c * 8);
-                const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
-                const float w = dw[j];
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        for (int j0 = 0; j0 < k; j0 += BATCH) {
+            uint4 v[BATCH];
+            float wj[BATCH];
+            bool ok[BATCH];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    acc[2 * m] = __fadd_rn(acc[2 * m], __fmul_rn(w, bf16_lo(pk[m])));
-                    acc[2 * m + 1] = __fadd_rn(acc[2 * m + 1], __fmul_rn(w, bf16_hi(pk[m])));
+            for (int u = 0; u < BATCH; ++u) {
+                const int j = j0 + u;
+                const int q = j < k ? __ldg(r.pair_rank + (size_t)t * k + j) : -1;
+                ok[u] = q >= 0;
+                wj[u] = ok[u] ? __ldg(r.topk_w + (size_t)t * k + j) : 0.0f;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (ok[u]) {
+                    const uint16_t *yq = static_cast<const uint16_t *>(g.y[q]);
+                    const size_t row = (size_t)__ldg(r.pair_row + (size_t)t * k + j);
+                    v[u] = ld_stream(yq + row * H + (size_t)c * 8);
                 }
             }
-            uint4 o;
-            o.x = pack_bf16x2(acc[0], acc[1]);
-            o.y = pack_bf16x2(acc[2], acc[3]);
-            o.z = pack_bf16x2(acc[4], acc[5]);
-            o.w = pack_bf16x2(acc[6], acc[7]);
-            *reinterpret_cast<uint4 *>(out + (size_t)t * H + (size_t)c * 8) = o;
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                if (!ok[u]) continue;
+                const uint32_t pk[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    acc[2 * m] = __fadd_rn(acc[2 * m], __fmul_rn(wj[u], bf16_lo(pk[m])));
+                    acc[2 * m + 1] = __fadd_rn(acc[2 * m + 1], __fmul_rn(wj[u], bf16_hi(pk[m])));
+                }
+            }
         }
-        __syncthreads();
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4 *>(out + (size_t)t * H + (size_t)c * 8) = o;
     }
 }
 
@@ -354,10 +358,13 @@ ep_status check_group(const ep_peer_group &g, const ep_peer_rank *ranks, bool ne
     return EP_OK;
 }
 
-int peer_blocks_per_rank(int n_local, int T_hint)
+// blocks per local rank: the GPU's resident blocks shared out over the local
+// ranks, and no more than the largest rank's chunks need
+int peer_blocks_per_rank(int n_local, int max_T, int chunks_per_row)
 {
-    int b = (device_sm_count() * 2 + n_local - 1) / n_local;
-    if (T_hint > 0 && b > T_hint) b = T_hint;
+    int b = (device_sm_count() * 8 + n_local - 1) / n_local;
+    const long long need = ((long long)max_T * chunks_per_row + PEER_THREADS - 1) / PEER_THREADS;
+    if (need < b) b = (int)need;
     return b < 1 ? 1 : b;
 }
 
@@ -368,16 +375,18 @@ using namespace ep;
 
 extern "C" {
 
-ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, ep_stream_t stream)
+ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, ep_stream_t stream)
 {
     const ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
-    const size_t smem = sizeof(int) * 2 * (size_t)g.P;
+    if (k < 1) return EP_ERR_INVALID;
+    if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    const size_t smem = sizeof(int) * (4 * (size_t)g.P + 1);
     if (smem > 48 * 1024)
         cudaFuncSetAttribute(peer_counts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     return launch_pdl(peer_counts_kernel, dim3(g.n_local), dim3(PEER_THREADS), smem,
-                      reinterpret_cast<cudaStream_t>(stream), g, ranks, wait_limit()) == cudaSuccess
+                      reinterpret_cast<cudaStream_t>(stream), g, ranks, k, wait_limit()) == cudaSuccess
                ? EP_OK
                : EP_ERR_CUDA;
 }
@@ -390,12 +399,8 @@ ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, in
     if (H < 128 || H % 128 != 0 || k < 1 || max_T < 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if (!g.recv_x || !g.recv_scale) return EP_ERR_INVALID;
-    const int bpr = peer_blocks_per_rank(g.n_local, max_T);
-    const size_t smem = sizeof(int) * (2 * (size_t)g.P + 1);
-    if (smem > 48 * 1024)
-        cudaFuncSetAttribute(peer_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    return launch_pdl(peer_dispatch_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), smem,
+    const int bpr = peer_blocks_per_rank(g.n_local, max_T, H / 16);
+    return launch_pdl(peer_dispatch_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), 0,
                       reinterpret_cast<cudaStream_t>(stream), g, ranks, H, k, bpr) == cudaSuccess
                ? EP_OK
                : EP_ERR_CUDA;
@@ -429,12 +434,8 @@ ep_status ep_peer_combine(ep_peer_group g, const ep_peer_rank *ranks, int H, int
     if (H < 8 || H % 8 != 0 || k < 1 || max_T < 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if (!g.y) return EP_ERR_INVALID;
-    const int bpr = peer_blocks_per_rank(g.n_local, max_T);
-    const size_t smem = sizeof(int) * (2 * (size_t)g.P + 1);
-    if (smem > 48 * 1024)
-        cudaFuncSetAttribute(peer_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    return launch_pdl(peer_combine_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), smem,
+    const int bpr = peer_blocks_per_rank(g.n_local, max_T, H / 8);
+    return launch_pdl(peer_combine_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), 0,
                       reinterpret_cast<cudaStream_t>(stream), g, ranks, H, k, bpr,
                       wait_limit()) == cudaSuccess
                ? EP_OK

@@ -64,7 +64,8 @@ class EpPath:
         self.dev_status = torch.zeros(1, **i32)    # layout (cleared by each layout call)
         self.copy_status = torch.zeros(1, **i32)   # dispatch / combine (sticky)
         ws = B.ep_workspace_size(T, k, P, R)
-        self.workspace = torch.empty(max(ws, 256), device=dev, dtype=torch.uint8)
+        # zeroed once: ep_route_dispatch keeps its counters there
+        self.workspace = torch.zeros(max(ws, 256), device=dev, dtype=torch.uint8)
         n = self.n_recv
         if self.fp8:
             self.recv_x = torch.empty((n, H), device=dev, dtype=torch.float8_e4m3fn)

@@ -101,7 +101,8 @@ typedef struct {
 /*
  * Bytes of device scratch that ep_dispatch_layout needs for T tokens, top-k,
  * P physical experts and R logical ranks (the counterpart of DeepEP's buffer
- * size hint).  Returns 0 for invalid sizes.  The scratch need not be zeroed.
+ * size hint).  Returns 0 for invalid sizes.  The scratch need not be zeroed
+ * for the layout calls; ep_route_dispatch wants it zeroed once (see there).
  */
 size_t ep_workspace_size(int T, int k, int P, int R);
 
@@ -236,8 +237,11 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
  *
  *   num_sms     SMs to use (0 = all): caps the fused kernel's blocks and the
  *               dispatch grid
- *   workspace   ep_workspace_size(T, k, P, R) bytes, 256-byte aligned; need
- *               not be zeroed (the call clears the words it counts on)
+ *   workspace   ep_workspace_size(T, k, P, R) bytes, 256-byte aligned.
+ *               Zero it once before its first use by this call: the fused
+ *               kernel counts on 16 bytes of it, and leaves them zero again
+ *               when it finishes (after a timeout too), so later calls need
+ *               no clearing; the other calls do not touch those bytes.
  *   dev_status  int32 [1] or NULL: zeroed by this call, then the layout's
  *               EP_DEV_BAD_* bits and EP_DEV_TIMEOUT if a bounded wait (for a
  *               TMA copy or for the other blocks) gave up, in which case the
@@ -501,12 +505,15 @@ typedef struct {
     int32_t *recv_cnt;          /* [P/W, W] (out): pairs from each source for each of
                                    this rank's experts (for its grouped GEMM) */
     int32_t *recv_rows;         /* [1] (out): rows this rank receives, padding included */
+    int32_t *pair_rank;         /* [T, k] (out): rank holding pair (t, j)'s row, -1 if none */
+    int32_t *pair_row;          /* [T, k] (out): that row */
     int32_t *dev_status;        /* [1] or NULL: EP_DEV_* bits are ORed in */
     int T;                      /* tokens of this rank */
     int reserved;
 } ep_peer_rank;
 
-ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, ep_stream_t stream);
+/* k: experts per token (the layouts' top-k), as for the calls below. */
+ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, ep_stream_t stream);
 /* H % 128 == 0; k <= 32; max_T: the largest T of the local ranks (sizes the grid). */
 ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, int k,
                            int max_T, ep_stream_t stream);

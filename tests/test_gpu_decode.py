@@ -209,7 +209,26 @@ def test_waits_give_up_and_report():
     finally:
         ep_testing_set_wait_limit(-1)
     assert int(path.dev_status.item()) & EP_DEV_TIMEOUT
+    # the same workspace: the calls that gave up left its counters clear
+    path.recv_x.view(torch.uint8).fill_(SENTINEL)
+    path.recv_scale.fill_(-7.0)
+    path.route_dispatch(lg, bias, x)
+    torch.cuda.synchronize()
+    check_against_oracle(cfg, wl, path)
+
+
+def test_workspace_shared_with_the_layout_calls():
+    """the route + layout calls (small-batch kernel and multi-tile kernels)
+    between two fused calls on one workspace leave its counters alone"""
+    cfg = CONFIGS["v3_decode"]
+    wl = Workload(cfg, seed=43)
     path = fresh_path(cfg, wl)
+    lg, bias, x = wl.logits.cuda(), wl.bias.cuda(), wl.x.cuda()
+    path.route_dispatch(lg, bias, x)
+    path.route_layout(lg, bias)
+    path.layout()
+    path.recv_x.view(torch.uint8).fill_(SENTINEL)
+    path.recv_scale.fill_(-7.0)
     path.route_dispatch(lg, bias, x)
     torch.cuda.synchronize()
     check_against_oracle(cfg, wl, path)
