@@ -63,8 +63,8 @@ class PeerRank(ctypes.Structure):
                 ("expert_off", ctypes.c_void_p), ("slot", ctypes.c_void_p),
                 ("topk_w", ctypes.c_void_p), ("out", ctypes.c_void_p),
                 ("dest_off", ctypes.c_void_p), ("recv_cnt", ctypes.c_void_p),
-                ("recv_rows", ctypes.c_void_p), ("pair_rank", ctypes.c_void_p),
-                ("pair_row", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
+                ("recv_rows", ctypes.c_void_p), ("pair_dest", ctypes.c_void_p),
+                ("dev_status", ctypes.c_void_p),
                 ("T", ctypes.c_int), ("reserved", ctypes.c_int)]
 
 

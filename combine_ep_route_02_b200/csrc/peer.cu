@@ -135,7 +135,8 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
     if (!ok_sh) {
         // no destination rows: the dispatch and combine skip every pair
         for (int p = tid; p < P; p += PEER_THREADS) r.dest_off[p] = -1;
-        for (int i = tid; i < r.T * k; i += PEER_THREADS) r.pair_rank[i] = -1;
+        for (int i = tid; i < r.T * k; i += PEER_THREADS)
+            reinterpret_cast<int2 *>(r.pair_dest)[i] = make_int2(-1, 0);
         if (tid == 0) {
             *r.recv_rows = 0;
             report(r, PEER_TIMEOUT);
@@ -180,8 +181,7 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
             overflow = PEER_OVERFLOW;
             q = -1;
         }
-        r.pair_rank[i] = q;
-        r.pair_row[i] = row;
+        reinterpret_cast<int2 *>(r.pair_dest)[i] = make_int2(q, row);
     }
     if (overflow) report(r, overflow);
 }
@@ -195,13 +195,23 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
 __global__ void __launch_bounds__(PEER_THREADS)
 peer_dispatch_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int bpr)
 {
+    extern __shared__ __align__(16) unsigned char psm[];
     __shared__ int last_sh;
     const int W = g.world;
     const int l = blockIdx.x / bpr, part = blockIdx.x % bpr, me = g.rank0 + l;
     const int tid = threadIdx.x;
     const ep_peer_rank &r = ranks[l];
+    // the ranks' receive rows and scales, as this process addresses them
+    uint8_t **rx = reinterpret_cast<uint8_t **>(psm);
+    float **rs = reinterpret_cast<float **>(psm) + W;
+    for (int q = tid; q < W; q += PEER_THREADS) {
+        rx[q] = static_cast<uint8_t *>(g.recv_x[q]);
+        rs[q] = g.recv_scale[q];
+    }
+    __syncthreads();
     pdl_launch_dependents();
     pdl_wait();
+    const int2 *pd = reinterpret_cast<const int2 *>(r.pair_dest);
     const int S = H >> 7, cpr = H >> 4;  // cpr is a multiple of 8
     const uint16_t *x = static_cast<const uint16_t *>(r.x);
     const long long total = (long long)r.T * cpr;
@@ -221,12 +231,11 @@ peer_dispatch_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, i
         const uint4 qv = quant::quant_chunk(lo, hi, scale);
         if (active)
             for (int j = 0; j < k; ++j) {
-                const int q = __ldg(r.pair_rank + (size_t)t * k + j);
-                if (q < 0) continue;
-                const size_t row = (size_t)__ldg(r.pair_row + (size_t)t * k + j);
-                uint8_t *dst = static_cast<uint8_t *>(g.recv_x[q]) + row * H;
-                *reinterpret_cast<uint4 *>(dst + (size_t)c * 16) = qv;
-                if ((c & 7) == 0) g.recv_scale[q][row * S + (c >> 3)] = scale;
+                const int2 qr = pd[(size_t)t * k + j];
+                if (qr.x < 0) continue;
+                const size_t row = (size_t)qr.y;
+                *reinterpret_cast<uint4 *>(rx[qr.x] + row * H + (size_t)c * 16) = qv;
+                if ((c & 7) == 0) rs[qr.x][row * S + (c >> 3)] = scale;
             }
     }
     // this block's rows are visible everywhere before it counts itself done
@@ -281,11 +290,14 @@ __global__ void __launch_bounds__(PEER_THREADS)
 peer_combine_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int bpr,
                     uint32_t limit)
 {
+    extern __shared__ __align__(16) unsigned char psm[];
     __shared__ int ok_sh;
     const int W = g.world;
     const int l = blockIdx.x / bpr, part = blockIdx.x % bpr, me = g.rank0 + l;
     const int tid = threadIdx.x;
     const ep_peer_rank &r = ranks[l];
+    const uint16_t **ys = reinterpret_cast<const uint16_t **>(psm);  // [W]
+    for (int q = tid; q < W; q += PEER_THREADS) ys[q] = static_cast<const uint16_t *>(g.y[q]);
     pdl_launch_dependents();
     pdl_wait();
     if (tid == 0) {
@@ -299,6 +311,7 @@ peer_combine_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, in
     if (!ok_sh) return;
     constexpr int BATCH = 8;
     const int cpr = H >> 3;
+    const int2 *pd = reinterpret_cast<const int2 *>(r.pair_dest);
     uint16_t *out = static_cast<uint16_t *>(r.out);
     const long long total = (long long)r.T * cpr;
     const long long g0 = (long long)part * PEER_THREADS + tid;
@@ -315,15 +328,11 @@ peer_combine_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, in
 #pragma unroll
             for (int u = 0; u < BATCH; ++u) {
                 const int j = j0 + u;
-                const int q = j < k ? __ldg(r.pair_rank + (size_t)t * k + j) : -1;
-                ok[u] = q >= 0;
+                const int2 qr = j < k ? pd[(size_t)t * k + j] : make_int2(-1, 0);
+                ok[u] = qr.x >= 0;
                 wj[u] = ok[u] ? __ldg(r.topk_w + (size_t)t * k + j) : 0.0f;
-                v[u] = make_uint4(0, 0, 0, 0);
-                if (ok[u]) {
-                    const uint16_t *yq = static_cast<const uint16_t *>(g.y[q]);
-                    const size_t row = (size_t)__ldg(r.pair_row + (size_t)t * k + j);
-                    v[u] = ld_stream(yq + row * H + (size_t)c * 8);
-                }
+                v[u] = ok[u] ? ld_stream(ys[qr.x] + (size_t)qr.y * H + (size_t)c * 8)
+                             : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int u = 0; u < BATCH; ++u) {
@@ -400,7 +409,11 @@ ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, in
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if (!g.recv_x || !g.recv_scale) return EP_ERR_INVALID;
     const int bpr = peer_blocks_per_rank(g.n_local, max_T, H / 16);
-    return launch_pdl(peer_dispatch_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), 0,
+    const size_t smem = 2 * sizeof(void *) * (size_t)g.world;
+    if (smem > 48 * 1024)
+        cudaFuncSetAttribute(peer_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    return launch_pdl(peer_dispatch_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), smem,
                       reinterpret_cast<cudaStream_t>(stream), g, ranks, H, k, bpr) == cudaSuccess
                ? EP_OK
                : EP_ERR_CUDA;
@@ -435,7 +448,8 @@ ep_status ep_peer_combine(ep_peer_group g, const ep_peer_rank *ranks, int H, int
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if (!g.y) return EP_ERR_INVALID;
     const int bpr = peer_blocks_per_rank(g.n_local, max_T, H / 8);
-    return launch_pdl(peer_combine_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), 0,
+    const size_t smem = sizeof(void *) * (size_t)g.world;
+    return launch_pdl(peer_combine_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), smem,
                       reinterpret_cast<cudaStream_t>(stream), g, ranks, H, k, bpr,
                       wait_limit()) == cudaSuccess
                ? EP_OK

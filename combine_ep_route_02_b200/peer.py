@@ -54,8 +54,8 @@ class EpPeerRanks:
         self.dest_off = [torch.empty(P, **i32) for _ in paths]
         self.recv_cnt = [torch.empty((epr, W), **i32) for _ in paths]
         self.recv_rows = [torch.empty(1, **i32) for _ in paths]
-        self.pair_rank = [torch.empty((p.T, p.k), **i32) for p in paths]
-        self.pair_row = [torch.empty((p.T, p.k), **i32) for p in paths]
+        # (rank, row) of every pair, written by the counts step
+        self.pair_dest = [torch.empty((p.T, p.k, 2), **i32) for p in paths]
         self.status = [torch.zeros(1, **i32) for _ in paths]
 
     def _tables(self, recv_x_all, recv_scale_all, y_all, board_all, flags_all, dev):
@@ -78,8 +78,8 @@ class EpPeerRanks:
                                 p.expert_off.data_ptr(), p.slot.data_ptr(),
                                 p.topk_w.data_ptr(), outs[i].data_ptr(),
                                 self.dest_off[i].data_ptr(), self.recv_cnt[i].data_ptr(),
-                                self.recv_rows[i].data_ptr(), self.pair_rank[i].data_ptr(),
-                                self.pair_row[i].data_ptr(), self.status[i].data_ptr(),
+                                self.recv_rows[i].data_ptr(), self.pair_dest[i].data_ptr(),
+                                self.status[i].data_ptr(),
                                 p.T, 0)
         raw = np.frombuffer(bytes(arr), dtype=np.uint8)
         self.ranks_dev = torch.from_numpy(raw.copy()).to(self.t_flags.device)

@@ -505,8 +505,8 @@ typedef struct {
     int32_t *recv_cnt;          /* [P/W, W] (out): pairs from each source for each of
                                    this rank's experts (for its grouped GEMM) */
     int32_t *recv_rows;         /* [1] (out): rows this rank receives, padding included */
-    int32_t *pair_rank;         /* [T, k] (out): rank holding pair (t, j)'s row, -1 if none */
-    int32_t *pair_row;          /* [T, k] (out): that row */
+    int32_t *pair_dest;         /* [T, k, 2] (out): (rank, row) holding pair (t, j)'s
+                                   row, rank -1 if none; 8-byte aligned */
     int32_t *dev_status;        /* [1] or NULL: EP_DEV_* bits are ORed in */
     int T;                      /* tokens of this rank */
     int reserved;

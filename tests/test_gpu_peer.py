@@ -93,9 +93,9 @@ def run_and_check(cfgs, wls, W, A, grp=None, seed=0):
     epr = P // W
     for s in range(W):
         assert np.array_equal(grp.dest_off[s].cpu().numpy(), dest_off[s])
-        pr, pw = grp.pair_rank[s].cpu().numpy(), grp.pair_row[s].cpu().numpy()
+        pd = grp.pair_dest[s].cpu().numpy()
         for (t, j), s_loc in np.ndenumerate(lays[s]["slot"]):
-            assert (pr[t, j], pw[t, j]) == row_of(lays[s], dest_off[s], s_loc, epr)
+            assert tuple(pd[t, j]) == row_of(lays[s], dest_off[s], s_loc, epr)
         assert int(grp.recv_rows[s].item()) == recv_rows[s]
         assert np.array_equal(grp.recv_cnt[s].cpu().numpy(), C[:, s * epr:(s + 1) * epr].T)
     # every destination row holds the oracle's row of its source
