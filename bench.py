@@ -627,9 +627,11 @@ def main():
         for i, yq in enumerate(grp.y):
             yq.copy_(device_normal_bf16(grp.cap, pcfg.H, seed=2000 + i))
         Kp = max(3, min(K, 50))
-        q0, q1, q2, q3 = (events(Kp) for _ in range(4))
+        qc, q0, q1, q2, q3 = (events(Kp) for _ in range(5))
         for i in range(args.warmup + Kp):
             j = i - args.warmup
+            if j >= 0:
+                qc[j].record(stream)
             grp.counts()
             if j >= 0:
                 q0[j].record(stream)
@@ -646,11 +648,12 @@ def main():
         torch.cuda.synchronize()
         if any(grp.check_status()):
             raise RuntimeError(f"peer step status {grp.check_status()}")
+        pn_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(qc, q0))
         pd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(q0, q1))
         pc_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(q2, q3))
         pab = algorithmic_bytes(pcfg)
         pd_bytes, pc_bytes = pab["dispatch"] * Wp, pab["combine"] * Wp
-        peer = {"ranks": Wp, "tokens_per_rank": pcfg.T,
+        peer = {"ranks": Wp, "tokens_per_rank": pcfg.T, "counts_us": pn_ms * 1e3,
                 "dispatch_us": pd_ms * 1e3, "dispatch_gbs": pd_bytes / (pd_ms * 1e-3) / 1e9,
                 "combine_us": pc_ms * 1e3, "combine_gbs": pc_bytes / (pc_ms * 1e-3) / 1e9,
                 "dispatch_combine_tokens_per_s": cfg.T / ((pd_ms + pc_ms) * 1e-3),

@@ -113,7 +113,7 @@ def lib() -> ctypes.CDLL:
         L.ep_combine_exchange.argtypes = [P, P, P, P, Z, P, P]
         L.ep_combine_exchange.restype = I
         G, RP = PeerGroup, ctypes.c_void_p
-        L.ep_peer_counts.argtypes = [G, RP, I, P]
+        L.ep_peer_counts.argtypes = [G, RP, I, I, P]
         L.ep_peer_counts.restype = I
         L.ep_peer_dispatch.argtypes = [G, RP, I, I, I, P]
         L.ep_peer_dispatch.restype = I
@@ -258,9 +258,10 @@ def ep_combine_exchange(comm: int, expert_rows, recv_rows, send_rows, row_bytes:
         _stream(stream)))
 
 
-def ep_peer_counts(group: PeerGroup, ranks_dev, k, stream=None):
+def ep_peer_counts(group: PeerGroup, ranks_dev, k, max_T, stream=None):
     """ranks_dev: device buffer holding n_local PeerRank structs."""
-    _check("ep_peer_counts", lib().ep_peer_counts(group, _ptr(ranks_dev), k, _stream(stream)))
+    _check("ep_peer_counts", lib().ep_peer_counts(group, _ptr(ranks_dev), k, max_T,
+                                                  _stream(stream)))
 
 
 def ep_peer_dispatch(group: PeerGroup, ranks_dev, H, k, max_T, stream=None):

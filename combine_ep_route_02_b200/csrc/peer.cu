@@ -101,7 +101,7 @@ EP_DEV void pair_dest(const int *eoff, const int *doff, int P, int epr, int s_lo
 // 1. all-gather of the per-expert counts, then this rank's destination
 //    offsets and receive counts.  One block per local rank.
 __global__ void __launch_bounds__(PEER_THREADS)
-peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t limit)
+peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
 {
     extern __shared__ int sm[];
     __shared__ int warp_tot[PEER_THREADS / 32 + 1];
@@ -111,8 +111,6 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
     const ep_peer_rank &r = ranks[l];
     int *tot = sm;            // [P] padded totals over all sources, then their scan
     int *pre = sm + P;        // [P] rows of sources before this one
-    int *eoff = sm + 2 * P;   // [P + 1] this rank's local expert offsets
-    int *doff = eoff + P + 1; // [P] destination offsets
     int32_t *my_flags = g.flags[me];
 
     pdl_launch_dependents();
@@ -135,8 +133,6 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
     if (!ok_sh) {
         // no destination rows: the dispatch and combine skip every pair
         for (int p = tid; p < P; p += PEER_THREADS) r.dest_off[p] = -1;
-        for (int i = tid; i < r.T * k; i += PEER_THREADS)
-            reinterpret_cast<int2 *>(r.pair_dest)[i] = make_int2(-1, 0);
         if (tid == 0) {
             *r.recv_rows = 0;
             report(r, PEER_TIMEOUT);
@@ -163,18 +159,32 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, uint32_t l
     const int total = layout_impl::block_exclusive_scan<PEER_THREADS>(tot, P, warp_tot);
     for (int p = tid; p < P; p += PEER_THREADS) {
         const int q = p / epr;
-        doff[p] = tot[p] - tot[q * epr] + pre[p];
-        r.dest_off[p] = doff[p];
+        r.dest_off[p] = tot[p] - tot[q * epr] + pre[p];
     }
-    for (int p = tid; p <= P; p += PEER_THREADS) eoff[p] = r.expert_off[p];
     if (tid == 0) {
         const int end = me + 1 < W ? tot[(me + 1) * epr] : total;
         *r.recv_rows = end - tot[me * epr];
     }
+}
+
+// 1b. every pair's destination rank and row, for the dispatch and combine.
+//     Grid: n_local x bpr blocks, a thread per pair.
+__global__ void __launch_bounds__(PEER_THREADS)
+peer_pairs_kernel(ep_peer_group g, const ep_peer_rank *ranks, int k, int bpr)
+{
+    extern __shared__ int sm[];
+    const int P = g.P, epr = P / g.world;
+    const int l = blockIdx.x / bpr, part = blockIdx.x % bpr, tid = threadIdx.x;
+    const ep_peer_rank &r = ranks[l];
+    int *eoff = sm;           // [P + 1] this rank's local expert offsets
+    int *doff = sm + P + 1;   // [P] destination offsets
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int p = tid; p <= P; p += PEER_THREADS) eoff[p] = r.expert_off[p];
+    for (int p = tid; p < P; p += PEER_THREADS) doff[p] = r.dest_off[p];
     __syncthreads();
-    // every pair's destination rank and row, for the dispatch and combine
     int overflow = 0;
-    for (int i = tid; i < r.T * k; i += PEER_THREADS) {
+    for (int i = part * PEER_THREADS + tid; i < r.T * k; i += bpr * PEER_THREADS) {
         int q, row;
         pair_dest(eoff, doff, P, epr, r.slot[i], q, row);
         if (q >= 0 && row >= g.cap) {
@@ -384,18 +394,30 @@ using namespace ep;
 
 extern "C" {
 
-ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, ep_stream_t stream)
+ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, int max_T,
+                         ep_stream_t stream)
 {
     const ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
-    if (k < 1) return EP_ERR_INVALID;
+    if (k < 1 || max_T < 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
-    const size_t smem = sizeof(int) * (4 * (size_t)g.P + 1);
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t smem = sizeof(int) * 2 * (size_t)g.P;
     if (smem > 48 * 1024)
         cudaFuncSetAttribute(peer_counts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-    return launch_pdl(peer_counts_kernel, dim3(g.n_local), dim3(PEER_THREADS), smem,
-                      reinterpret_cast<cudaStream_t>(stream), g, ranks, k, wait_limit()) == cudaSuccess
+    if (launch_pdl(peer_counts_kernel, dim3(g.n_local), dim3(PEER_THREADS), smem, s, g, ranks,
+                   wait_limit()) != cudaSuccess)
+        return EP_ERR_CUDA;
+    // the pairs' destinations: a thread per pair of the largest rank
+    int bpr = (int)(((long long)max_T * k + PEER_THREADS - 1) / PEER_THREADS);
+    if (bpr < 1) bpr = 1;
+    const size_t smem2 = sizeof(int) * (2 * (size_t)g.P + 1);
+    if (smem2 > 48 * 1024)
+        cudaFuncSetAttribute(peer_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem2);
+    return launch_pdl(peer_pairs_kernel, dim3(g.n_local * bpr), dim3(PEER_THREADS), smem2, s, g,
+                      ranks, k, bpr) == cudaSuccess
                ? EP_OK
                : EP_ERR_CUDA;
 }

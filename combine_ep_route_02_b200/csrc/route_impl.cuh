@@ -224,13 +224,29 @@ EP_DEV int warp_pick(uint32_t key, int idx)
     return (int)__reduce_min_sync(FULL_MASK, cand);
 }
 
-// Routes tokens t_first, t_first + t_stride, ... < T with the calling warp.
-// tab: the 2^(j/64) table in shared memory.
+// Bias and token-invariant group id of each expert a lane holds (lane l
+// holds experts [l*EPL, (l+1)*EPL)); -1: no such expert.
 template <int EPL>
-EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restrict__ bias, int T,
-                         int E, int G, int Kg, int k, float scale, int renorm, int vec4,
-                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                         const double *tab, int t_first, int t_stride)
+EP_DEV void lane_experts(const float *__restrict__ bias, int E, int G, float (&b)[EPL],
+                         int (&gid)[EPL])
+{
+    const int e0 = (threadIdx.x & 31) * EPL;
+    const int gs = E / G;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const bool v = e0 + i < E;
+        b[i] = (bias != nullptr && v) ? bias[e0 + i] : 0.0f;
+        gid[i] = v ? (e0 + i) / gs : -1;
+    }
+}
+
+// Selection for token t from its sigmoids s (the lane layout above; 0 for
+// experts past E): keys s + b, group scores and the kept groups, the k
+// largest keys, the weights; writes row t of topk_idx and topk_w.
+template <int EPL>
+EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)[EPL], int E,
+                        int G, int Kg, int k, float scale, int renorm,
+                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int t)
 {
     const int lane = threadIdx.x & 31;
     const int e0 = lane * EPL;
@@ -241,15 +257,159 @@ EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restri
     const bool aligned = (gs % EPL) == 0 && (lpg & (lpg - 1)) == 0;
     const int lanes_per_group = aligned ? lpg : 0;
     const int my_group = (e0 < E) ? e0 / gs : -1;        // valid when aligned
-
-    float b[EPL];
-    int gid[EPL];  // token-invariant group of each held expert (-1: none)
+    uint32_t key[EPL];
+    uint32_t live = 0;  // bit i: expert e0+i exists and is still eligible
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-        const bool v = e0 + i < E;
-        b[i] = (bias != nullptr && v) ? bias[e0 + i] : 0.0f;
-        gid[i] = v ? (e0 + i) / gs : -1;
+        if (e0 + i < E) {
+            key[i] = ordered(__fadd_rn(__fadd_rn(s[i], b[i]), 0.0f));
+            live |= 1u << i;
+        } else {
+            key[i] = NONE;
+        }
     }
+
+    if (G > 1) {
+        // group score = fp32 sum of the two largest keys in the group
+        uint32_t chosen = 0;
+        if (aligned) {
+            float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                if (!((live >> i) & 1u)) continue;
+                const float v = __fadd_rn(s[i], b[i]);
+                if (v > a1) {
+                    a2 = a1;
+                    a1 = v;
+                } else if (v > a2) {
+                    a2 = v;
+                }
+            }
+            // butterfly over the lanes of this group (they are contiguous
+            // and start at a multiple of lanes_per_group)
+            for (int off = 1; off < lanes_per_group; off <<= 1) {
+                const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                a1 = fmaxf(a1, o1);
+                a2 = n2;
+            }
+            const uint32_t my_score =
+                (my_group >= 0) ? ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f)) : NONE;
+            for (int r = 0; r < Kg; ++r) {
+                const bool cand = my_group >= 0 && !((chosen >> my_group) & 1u);
+                const int g = warp_pick(cand ? my_score : NONE, cand ? my_group : 0x7fffffff);
+                chosen |= 1u << g;
+            }
+        } else {
+            uint32_t my_score = NONE;  // lane g keeps the score of group g
+            for (int g = 0; g < G; ++g) {
+                float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) {
+                    if (gid[i] != g) continue;
+                    const float v = __fadd_rn(s[i], b[i]);
+                    if (v > a1) {
+                        a2 = a1;
+                        a1 = v;
+                    } else if (v > a2) {
+                        a2 = v;
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
+                    const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
+                    const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
+                    a1 = fmaxf(a1, o1);
+                    a2 = n2;
+                }
+                if (lane == g) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
+            }
+            for (int r = 0; r < Kg; ++r) {
+                const bool cand = lane < G && !((chosen >> lane) & 1u);
+                const int g = warp_pick(cand ? my_score : NONE, cand ? lane : 0x7fffffff);
+                chosen |= 1u << g;
+            }
+        }
+        if (aligned) {
+            // the lane's experts share one group
+            if (my_group >= 0 && !((chosen >> my_group) & 1u))
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) key[i] = NONE;
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) key[i] = NONE;
+        }
+    }
+
+    // lane-local best: the first (lowest index) of the largest keys;
+    // excluded and taken experts hold NONE, below every real key
+    uint32_t best_k = NONE;
+    int best_i = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (key[i] > best_k) {
+            best_k = key[i];
+            best_i = e0 + i;
+        }
+
+    int sel_idx = 0;
+    float sel_s = 0.0f;
+    for (int r = 0; r < k; ++r) {
+        const int e = warp_pick(best_k, best_i);
+        const int owner = e / EPL;  // k <= eligible experts, so e is real
+        float sv = 0.0f;
+        if (lane == owner) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (e0 + i == e) {
+                    sv = s[i];
+                    key[i] = NONE;
+                }
+            best_k = NONE;
+            best_i = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (key[i] > best_k) {
+                    best_k = key[i];
+                    best_i = e0 + i;
+                }
+        }
+        sv = __shfl_sync(FULL_MASK, sv, owner);
+        if (lane == r) {
+            sel_idx = e;
+            sel_s = sv;
+        }
+    }
+
+    float w = sel_s;
+    if (renorm) {
+        float sum = 0.0f;
+        for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(FULL_MASK, sel_s, j));
+        if (sum != 0.0f) w = __fdiv_rn(w, sum);
+    }
+    w = __fmul_rn(w, scale);
+    if (lane < k) {
+        topk_idx[(size_t)t * k + lane] = sel_idx;
+        topk_w[(size_t)t * k + lane] = w;
+    }
+}
+
+// Routes tokens t_first, t_first + t_stride, ... < T with the calling warp.
+// tab: the 2^(j/64) table in shared memory.
+template <int EPL>
+EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restrict__ bias, int T,
+                         int E, int G, int Kg, int k, float scale, int renorm, int vec4,
+                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                         const double *tab, int t_first, int t_stride)
+{
+    const int lane = threadIdx.x & 31;
+    const int e0 = lane * EPL;
+    float b[EPL];
+    int gid[EPL];
+    lane_experts<EPL>(bias, E, G, b, gid);
 
     for (int t = t_first; t < T; t += t_stride) {
         const float *row = logits + (size_t)t * E;
@@ -271,10 +431,8 @@ EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restri
             for (int i = 0; i < EPL; ++i) x[i] = (e0 + i < E) ? __ldg(row + e0 + i) : 0.0f;
         }
 
-        // s = the exact sigmoid rounded to fp32; key = fp32(s + b)
+        // s = the exact sigmoid rounded to fp32
         float s[EPL];
-        uint32_t key[EPL];
-        uint32_t live = 0;  // bit i: expert e0+i exists and is still eligible
         uint32_t near = 0;  // bit i: s[i] needs the exact evaluation
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
@@ -287,142 +445,7 @@ EP_DEV void route_tokens(const float *__restrict__ logits, const float *__restri
             for (int i = 0; i < EPL; ++i)
                 if ((near >> i) & 1u) s[i] = sigmoid_exact(x[i]);
         }
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            if (e0 + i < E) {
-                key[i] = ordered(__fadd_rn(__fadd_rn(s[i], b[i]), 0.0f));
-                live |= 1u << i;
-            } else {
-                key[i] = NONE;
-            }
-        }
-
-        if (G > 1) {
-            // group score = fp32 sum of the two largest keys in the group
-            uint32_t chosen = 0;
-            if (aligned) {
-                float a1 = -INFINITY, a2 = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i) {
-                    if (!((live >> i) & 1u)) continue;
-                    const float v = __fadd_rn(s[i], b[i]);
-                    if (v > a1) {
-                        a2 = a1;
-                        a1 = v;
-                    } else if (v > a2) {
-                        a2 = v;
-                    }
-                }
-                // butterfly over the lanes of this group (they are contiguous
-                // and start at a multiple of lanes_per_group)
-                for (int off = 1; off < lanes_per_group; off <<= 1) {
-                    const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
-                    const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
-                    const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
-                    a1 = fmaxf(a1, o1);
-                    a2 = n2;
-                }
-                const uint32_t my_score =
-                    (my_group >= 0) ? ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f)) : NONE;
-                for (int r = 0; r < Kg; ++r) {
-                    const bool cand = my_group >= 0 && !((chosen >> my_group) & 1u);
-                    const int g = warp_pick(cand ? my_score : NONE, cand ? my_group : 0x7fffffff);
-                    chosen |= 1u << g;
-                }
-            } else {
-                uint32_t my_score = NONE;  // lane g keeps the score of group g
-                for (int g = 0; g < G; ++g) {
-                    float a1 = -INFINITY, a2 = -INFINITY;
-#pragma unroll
-                    for (int i = 0; i < EPL; ++i) {
-                        if (gid[i] != g) continue;
-                        const float v = __fadd_rn(s[i], b[i]);
-                        if (v > a1) {
-                            a2 = a1;
-                            a1 = v;
-                        } else if (v > a2) {
-                            a2 = v;
-                        }
-                    }
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) {
-                        const float o1 = __shfl_xor_sync(FULL_MASK, a1, off);
-                        const float o2 = __shfl_xor_sync(FULL_MASK, a2, off);
-                        const float n2 = (a1 >= o1) ? fmaxf(a2, o1) : fmaxf(a1, o2);
-                        a1 = fmaxf(a1, o1);
-                        a2 = n2;
-                    }
-                    if (lane == g) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
-                }
-                for (int r = 0; r < Kg; ++r) {
-                    const bool cand = lane < G && !((chosen >> lane) & 1u);
-                    const int g = warp_pick(cand ? my_score : NONE, cand ? lane : 0x7fffffff);
-                    chosen |= 1u << g;
-                }
-            }
-            if (aligned) {
-                // the lane's experts share one group
-                if (my_group >= 0 && !((chosen >> my_group) & 1u))
-#pragma unroll
-                    for (int i = 0; i < EPL; ++i) key[i] = NONE;
-            } else {
-#pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (gid[i] >= 0 && !((chosen >> gid[i]) & 1u)) key[i] = NONE;
-            }
-        }
-
-        // lane-local best: the first (lowest index) of the largest keys;
-        // excluded and taken experts hold NONE, below every real key
-        uint32_t best_k = NONE;
-        int best_i = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i)
-            if (key[i] > best_k) {
-                best_k = key[i];
-                best_i = e0 + i;
-            }
-
-        int sel_idx = 0;
-        float sel_s = 0.0f;
-        for (int r = 0; r < k; ++r) {
-            const int e = warp_pick(best_k, best_i);
-            const int owner = e / EPL;  // k <= eligible experts, so e is real
-            float sv = 0.0f;
-            if (lane == owner) {
-#pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (e0 + i == e) {
-                        sv = s[i];
-                        key[i] = NONE;
-                    }
-                best_k = NONE;
-                best_i = 0x7fffffff;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (key[i] > best_k) {
-                        best_k = key[i];
-                        best_i = e0 + i;
-                    }
-            }
-            sv = __shfl_sync(FULL_MASK, sv, owner);
-            if (lane == r) {
-                sel_idx = e;
-                sel_s = sv;
-            }
-        }
-
-        float w = sel_s;
-        if (renorm) {
-            float sum = 0.0f;
-            for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(FULL_MASK, sel_s, j));
-            if (sum != 0.0f) w = __fdiv_rn(w, sum);
-        }
-        w = __fmul_rn(w, scale);
-        if (lane < k) {
-            topk_idx[(size_t)t * k + lane] = sel_idx;
-            topk_w[(size_t)t * k + lane] = w;
-        }
+        select_topk<EPL>(s, b, gid, E, G, Kg, k, scale, renorm, topk_idx, topk_w, t);
     }
 }
 

@@ -88,7 +88,7 @@ class EpPeerRanks:
 
     # the step ---------------------------------------------------------
     def counts(self, stream=None):
-        B.ep_peer_counts(self.group, self.ranks_dev, self.k, stream)
+        B.ep_peer_counts(self.group, self.ranks_dev, self.k, self.max_T, stream)
 
     def dispatch(self, stream=None):
         B.ep_peer_dispatch(self.group, self.ranks_dev, self.H, self.k, self.max_T, stream)

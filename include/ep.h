@@ -512,8 +512,10 @@ typedef struct {
     int reserved;
 } ep_peer_rank;
 
-/* k: experts per token (the layouts' top-k), as for the calls below. */
-ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, ep_stream_t stream);
+/* k: experts per token (the layouts' top-k); max_T: the largest T of the
+ * local ranks.  Also writes every local pair's (rank, row) in pair_dest. */
+ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, int max_T,
+                         ep_stream_t stream);
 /* H % 128 == 0; k <= 32; max_T: the largest T of the local ranks (sizes the grid). */
 ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, int k,
                            int max_T, ep_stream_t stream);

@@ -125,6 +125,16 @@ def run_and_check(cfgs, wls, W, A, grp=None, seed=0):
     return grp
 
 
+def test_peer_step_other_shape():
+    """the DeepSeek-16B shape (64 experts without groups, top-6, H = 2048)
+    over 4 ranks with a 32-row tile, ranks of very different sizes"""
+    W, A = 4, 32
+    base = CONFIGS["ds16b"]
+    cfgs = [dataclasses.replace(base.scaled(T), R=W) for T in (1, 300, 57, 512)]
+    wls = [Workload(c, seed=90 + r) for r, c in enumerate(cfgs)]
+    run_and_check(cfgs, wls, W, A, seed=4)
+
+
 @pytest.mark.parametrize("W,A", [(4, 1), (4, 16), (8, 1)])
 def test_peer_step_matches_oracle(W, A):
     """DeepSeek-V3 routing (256 experts, 8 groups, top-8) over W ranks, a
