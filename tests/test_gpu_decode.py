@@ -104,6 +104,30 @@ def test_other_shapes(name, T):
     check_against_oracle(cfg, wl, path)
 
 
+@pytest.mark.parametrize("R", [128, 256])
+def test_many_ranks(R):
+    """128 and 256 logical ranks (tokens per rank counted by a warp per rank,
+    shared out over the blocks)"""
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS["v3_decode"].scaled(200), R=R)
+    wl = Workload(cfg, seed=R)
+    path = run_fused(cfg, wl)
+    assert path.fused_route_dispatch()
+    check_against_oracle(cfg, wl, path)
+
+
+def test_largest_instance():
+    """1024 experts in 32 groups, 8 kept, top-32 (the kernel instance with 32
+    experts per lane), H = 512, with a 64-row tile"""
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS["v3_decode"].scaled(100), H=512, E=1024, R=16,
+                              n_group=32, topk_group=8, topk=32)
+    wl = Workload(cfg, seed=7)
+    path = run_fused(cfg, wl, row_align=64)
+    assert path.fused_route_dispatch()
+    check_against_oracle(cfg, wl, path, row_align=64)
+
+
 @pytest.mark.parametrize("A", [16, 128])
 def test_gemm_layout(A):
     """each expert's rows start on a multiple of the row tile; padding rows
