@@ -122,9 +122,9 @@ peer_counts_kernel(ep_peer_group g, const ep_peer_rank *ranks, uint32_t limit)
     // this rank's counts into row `me` of every rank's board
     for (int q = 0; q < W; ++q)
         for (int p = tid; p < P; p += PEER_THREADS) g.board[q][(size_t)me * P + p] = r.cnt_expert[p];
-    __threadfence_system();
     __syncthreads();
     if (tid == 0) {
+        __threadfence_system();  // cumulative over the block's board stores
         for (int q = 0; q < W; ++q) red_release_sys(&g.flags[q][0], 1);
         ok_sh = wait_at_least(&my_flags[0], W * step_sh, limit);
         if (!ok_sh) my_flags[5] |= PEER_TIMEOUT;
@@ -248,10 +248,12 @@ peer_dispatch_kernel(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, i
                 if ((c & 7) == 0) rs[qr.x][row * S + (c >> 3)] = scale;
             }
     }
-    // this block's rows are visible everywhere before it counts itself done
-    __threadfence_system();
+    // this block's rows are visible everywhere before it counts itself
+    // done: the block's barrier orders its threads' stores before thread 0's
+    // system-scope fence, which is cumulative over them
     __syncthreads();
     if (tid == 0) {
+        __threadfence_system();
         const int done = atomicAdd(&g.flags[me][4], 1);
         last_sh = done == bpr - 1;
     }
