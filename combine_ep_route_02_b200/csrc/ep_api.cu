@@ -170,6 +170,7 @@ extern "C" {
 ep_status ep_route(const float *logits, const float *bias, int T, ep_route_cfg cfg,
                    int32_t *topk_idx, float *topk_w, ep_stream_t stream)
 {
+    EP_TRACE("ep_route");
     const ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
     if (st != EP_OK) return st;
     RouteArgs a{logits, bias, T, cfg.num_experts, cfg.n_group, cfg.topk_group, cfg.topk,
@@ -184,6 +185,7 @@ ep_status ep_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int P
                              uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
                              int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_dispatch_layout");
     const ep_status st = check_layout(topk_idx, T, k, E, P, R, phys_of, n_rep, max_rep, row_align,
                                       cnt_expert, expert_off, rows_rank, rank_off, tok_rank,
                                       in_rank, slot, src, workspace, dev_status);
@@ -202,6 +204,7 @@ ep_status ep_route_layout(const float *logits, const float *bias, int T, ep_rout
                           int32_t *tok_rank, uint8_t *in_rank, int32_t *slot, int32_t *src,
                           void *workspace, int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_route_layout");
     ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
     if (st != EP_OK) return st;
     const int E = cfg.num_experts, k = cfg.topk;
@@ -229,6 +232,7 @@ ep_status ep_dispatch(const void *x_bf16, int T, int H, int k, int recv_rows,
                       const int32_t *slot, int fp8, void *recv_x, float *recv_scale, int num_sms,
                       int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_dispatch");
     if (T < 0 || H < 1 || k < 1) return EP_ERR_INVALID;
     if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
@@ -253,6 +257,7 @@ ep_status ep_route_dispatch(const float *logits, const float *bias, int T, ep_ro
                             uint8_t *in_rank, int32_t *slot, int32_t *src, void *workspace,
                             int num_sms, int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_route_dispatch");
     ep_status st = check_route(logits, bias, T, cfg, topk_idx, topk_w);
     if (st != EP_OK) return st;
     const int E = cfg.num_experts, k = cfg.topk;
@@ -293,6 +298,7 @@ ep_status ep_route_dispatch(const float *logits, const float *bias, int T, ep_ro
 
 ep_status ep_testing_set_wait_limit(long long polls)
 {
+    EP_TRACE("ep_testing_set_wait_limit");
     if (polls > 0xffffffffLL) return EP_ERR_INVALID;
     g_wait_limit.store(polls < 0 ? -1 : polls, std::memory_order_relaxed);
     return EP_OK;
@@ -302,6 +308,7 @@ ep_status ep_combine(const void *y_bf16, const int32_t *slot, const float *topk_
                      int k, int recv_rows, void *out_bf16, int num_sms, int32_t *dev_status,
                      ep_stream_t stream)
 {
+    EP_TRACE("ep_combine");
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
@@ -318,6 +325,7 @@ ep_status ep_dispatch_backward(const void *grad_recv_bf16, const int32_t *slot, 
                                int k, int recv_rows, void *grad_x_bf16, int num_sms,
                                int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_dispatch_backward");
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
@@ -335,6 +343,7 @@ ep_status ep_combine_backward(const void *grad_out_bf16, const void *y_bf16, con
                               void *grad_y_bf16, float *grad_w, int num_sms, int32_t *dev_status,
                               ep_stream_t stream)
 {
+    EP_TRACE("ep_combine_backward");
     if (T < 0 || H < 1 || k < 1 || H % 8 != 0) return EP_ERR_INVALID;
     if (k > MAX_TOPK) return EP_ERR_UNSUPPORTED;
     if ((long long)T * k >= (1LL << 31) || T > (1 << 30)) return EP_ERR_UNSUPPORTED;
@@ -360,6 +369,7 @@ ep_status ep_silu_mul(const void *gate_up_bf16, int n_rows, int I, const int32_t
                       const int32_t *cnt_expert, int P, int fp8, void *act, float *act_scale,
                       int num_sms, ep_stream_t stream)
 {
+    EP_TRACE("ep_silu_mul");
     if (n_rows < 0 || I < 1 || I % 128 != 0) return EP_ERR_INVALID;
     if ((expert_off == nullptr) != (cnt_expert == nullptr)) return EP_ERR_INVALID;
     if (expert_off != nullptr && P < 1) return EP_ERR_INVALID;

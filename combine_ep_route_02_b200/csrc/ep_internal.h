@@ -3,9 +3,20 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace ep {
+
+// A named NVTX range around each entry point (shows up in Nsight Systems
+// timelines; without an attached tool the calls return at once).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+#define EP_TRACE(name) ::ep::NvtxRange ep_nvtx_range_(name)
 
 // Layout tiling.  A tile of tokens is one block of the count and slot
 // kernels.  Up to LAYOUT_FUSED_MAX_TILES tiles, the slot kernel sums the tile

@@ -132,6 +132,7 @@ ep_status ep_exchange_counts(ep_nccl_comm comm, const int32_t *rows_rank,
                              const int32_t *cnt_expert, int P, int32_t *send_scratch,
                              int32_t *recv_counts, ep_stream_t stream)
 {
+    EP_TRACE("ep_exchange_counts");
     const NcclApi *api = nccl();
     if (api == nullptr) return EP_ERR_UNSUPPORTED;
     if (comm == nullptr || !rows_rank || !cnt_expert || !send_scratch || !recv_counts || P < 1)
@@ -163,6 +164,7 @@ ep_status ep_dispatch_exchange(ep_nccl_comm comm, const void *rows, const int32_
                                const int32_t *recv_rows, size_t row_bytes, void *recv,
                                ep_stream_t stream)
 {
+    EP_TRACE("ep_dispatch_exchange");
     if (comm == nullptr) return EP_ERR_INVALID;
     return exchange_rows(reinterpret_cast<ncclComm_t>(comm), rows, send_rows, recv_rows,
                          row_bytes, recv, reinterpret_cast<cudaStream_t>(stream));
@@ -172,6 +174,7 @@ ep_status ep_combine_exchange(ep_nccl_comm comm, const void *expert_rows,
                               const int32_t *recv_rows, const int32_t *send_rows,
                               size_t row_bytes, void *back, ep_stream_t stream)
 {
+    EP_TRACE("ep_combine_exchange");
     if (comm == nullptr) return EP_ERR_INVALID;
     // the reverse direction: what arrived from rank q goes back to rank q
     return exchange_rows(reinterpret_cast<ncclComm_t>(comm), expert_rows, recv_rows, send_rows,

@@ -49,6 +49,7 @@ extern "C" ep_status ep_dispatch_layout_noalloc(
     int32_t *rows_rank, int32_t *rank_off, int32_t *tok_rank, uint8_t *in_rank, int32_t *slot,
     int32_t *src, int32_t *dev_status, ep_stream_t stream)
 {
+    EP_TRACE("ep_dispatch_layout_noalloc");
     const size_t need = ep_workspace_size(T, k, P, R);
     if (need == 0) return EP_ERR_INVALID;
     if (need > EP_NOALLOC_SCRATCH_BYTES) return EP_ERR_UNSUPPORTED;

@@ -399,6 +399,7 @@ extern "C" {
 ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, int max_T,
                          ep_stream_t stream)
 {
+    EP_TRACE("ep_peer_counts");
     const ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
     if (k < 1 || max_T < 0) return EP_ERR_INVALID;
@@ -427,6 +428,7 @@ ep_status ep_peer_counts(ep_peer_group g, const ep_peer_rank *ranks, int k, int 
 ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, int k,
                            int max_T, ep_stream_t stream)
 {
+    EP_TRACE("ep_peer_dispatch");
     ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
     if (H < 128 || H % 128 != 0 || k < 1 || max_T < 0) return EP_ERR_INVALID;
@@ -445,6 +447,7 @@ ep_status ep_peer_dispatch(ep_peer_group g, const ep_peer_rank *ranks, int H, in
 
 ep_status ep_peer_wait_dispatch(ep_peer_group g, const ep_peer_rank *ranks, ep_stream_t stream)
 {
+    EP_TRACE("ep_peer_wait_dispatch");
     const ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
     return launch_pdl(peer_wait_kernel, dim3(g.n_local), dim3(32), 0,
@@ -455,6 +458,7 @@ ep_status ep_peer_wait_dispatch(ep_peer_group g, const ep_peer_rank *ranks, ep_s
 
 ep_status ep_peer_experts_ready(ep_peer_group g, ep_stream_t stream)
 {
+    EP_TRACE("ep_peer_experts_ready");
     const ep_status st = check_group(g, nullptr, false);
     if (st != EP_OK) return st;
     return launch_pdl(peer_ready_kernel, dim3(g.n_local), dim3(32), 0,
@@ -466,6 +470,7 @@ ep_status ep_peer_experts_ready(ep_peer_group g, ep_stream_t stream)
 ep_status ep_peer_combine(ep_peer_group g, const ep_peer_rank *ranks, int H, int k, int max_T,
                           ep_stream_t stream)
 {
+    EP_TRACE("ep_peer_combine");
     ep_status st = check_group(g, ranks);
     if (st != EP_OK) return st;
     if (H < 8 || H % 8 != 0 || k < 1 || max_T < 0) return EP_ERR_INVALID;
