@@ -13,15 +13,17 @@
 //   h = bf16(fp32(s * u))
 //   then the dispatch quantiser on h (quant.cuh).
 // The correctly rounded SiLU is a function of the 16-bit gate pattern: a
-// table generated at build time (gen_silu_table.c, x87 extended precision)
-// holds it for the 8,192 gates with 2^-25 <= |g| < 2^7, and each block keeps
-// a copy in shared memory.  Outside that range it has closed forms (below:
-// g/2 with ties toward +inf; above: g for g > 0 and -0 for g < 0), taken only
-// by warps that meet such a gate.  Every one of the 65,536 bf16 gates is
-// checked against the oracle on the GPU.
+// table generated at build time (gen_silu_table.c) holds it for all 65,536
+// patterns, NaN, infinities and the closed-form ranges included, and each
+// block copies it (128 KB) into shared memory, where a lookup indexed by the
+// raw gate bits costs one shared load and no range test.  Every entry is
+// checked against the oracle on the host, and every gate through the kernel
+// on the GPU.
 //
-// Mapping: the filled rows are numbered v = 0 .. V-1 in expert order (V = sum
-// of the counts) and each block takes a contiguous range of them; a thread
+// Mapping: one block of 768 threads per SM (the table leaves room for one),
+// so 24 warps keep loads in flight.  The filled rows are numbered v = 0 ..
+// V-1 in expert order (V = sum of the counts) and each block takes a
+// contiguous range of them; a thread
 // owns a 16-element chunk of one output row (two 16-byte loads of gate, two
 // of up, one 16-byte store of e4m3), and the 8 lanes of a 128-element block
 // reduce its amax with shuffles.  Each block keeps the counts' prefix sum in
@@ -36,48 +38,14 @@ namespace ep {
 
 namespace {
 
-constexpr int ACT_THREADS = 256;
+constexpr int ACT_THREADS = 768;
 
-// silu(g) correctly rounded to bf16 for the gates with 2^-25 <= |g| < 2^7,
-// generated at build time (gen_silu_table.c): entry (sign << 12) | (|g|
-// pattern - 0x3300).
-constexpr uint32_t TAB_BASE = 0x3300u;  // |g| pattern of 2^-25
-constexpr int TAB_SIZE = 8192;
+// silu(g) correctly rounded to bf16 for every bf16 gate pattern g (entry g),
+// generated at build time (gen_silu_table.c).
+constexpr int TAB_SIZE = 65536;
 __device__ const uint16_t kSiluTable[TAB_SIZE] = {
 #include "silu_table.inc"
 };
-
-// silu of both gates of a packed bf16 pair w, as a packed bf16 pair, from
-// the table.  Each 16-bit half is offset with its bit 15 set as a guard, so
-// the subtraction never borrows across halves; a half is in the table's
-// range iff its top four bits come out as 1000.  `bad` gets nonzero bits
-// when a gate is outside the range (its entry is then unrelated).
-EP_DEV uint32_t silu_pair_table(uint32_t w, const uint16_t *tab, uint32_t &bad)
-{
-    const uint32_t d = ((w & 0x7FFF7FFFu) | 0x80008000u) - TAB_BASE * 0x10001u;
-    bad |= (d & 0xF000F000u) ^ 0x80008000u;
-    const uint32_t i_lo = (d & 0x0FFFu) | ((w >> 3) & 0x1000u);
-    const uint32_t i_hi = ((d >> 16) & 0x0FFFu) | ((w >> 19) & 0x1000u);
-    return __byte_perm((uint32_t)tab[i_lo], (uint32_t)tab[i_hi], 0x5410);
-}
-
-// silu(g) for any bf16 gate pattern b (low 16 bits), as a bf16 pattern: the
-// table inside its range, else the closed forms.  |g| < 2^-25: silu(g) - g/2
-// = g tanh(g/2) / 2 is positive and below half a bf16 step of g/2, so the
-// result is g/2 (exact in fp32) rounded to bf16 with ties toward +inf (a tie
-// occurs only below 2^-126).  |g| >= 2^7 and inf: g for g > 0, -0 for g < 0
-// (|g e^g| < 2^-180).  NaN: NaN.
-EP_DEV uint32_t silu_any(uint32_t b, const uint16_t *tab)
-{
-    const uint32_t a = b & 0x7FFFu;
-    if (a - TAB_BASE < 4096u) return tab[((b >> 3) & 0x1000u) | (a - TAB_BASE)];
-    if (a < TAB_BASE) {
-        const uint32_t h = __float_as_uint(__uint_as_float(b << 16) * 0.5f);
-        return ((h + ((h >> 31) ? 0x7FFFu : 0x8000u)) >> 16) & 0xFFFFu;
-    }
-    const bool neg_zero = (b & 0x8000u) && a <= 0x7F80u;
-    return neg_zero ? 0x8000u : b;
-}
 
 // bf16x2 product rounded once to nearest even.  s and u have 8-bit
 // significands, so s * u is exact in fp32 wherever bf16 rounding can give a
@@ -89,30 +57,20 @@ EP_DEV uint32_t mul_bf16x2(uint32_t a, uint32_t b)
     return r;
 }
 
-// h for the 8 elements of one 16-byte gate vector and one 16-byte up vector.
-// FULL = false: table lookups only, `bad` reports gates the table does not
-// cover (the caller then redoes the chunk with FULL = true).
-template <bool FULL>
-EP_DEV uint4 silu_mul8(uint4 g, uint4 u, const uint16_t *tab, uint32_t &bad)
+// h for the 8 elements of one 16-byte gate vector and one 16-byte up vector:
+// both halves of each packed gate pair index the table directly.
+EP_DEV uint4 silu_mul8(uint4 g, uint4 u, const uint16_t *tab)
 {
     const uint32_t gp[4] = {g.x, g.y, g.z, g.w};
     const uint32_t up[4] = {u.x, u.y, u.z, u.w};
     uint32_t h[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        const uint32_t s = FULL ? __byte_perm(silu_any(gp[m] & 0xFFFFu, tab),
-                                              silu_any(gp[m] >> 16, tab), 0x5410)
-                                : silu_pair_table(gp[m], tab, bad);
+        const uint32_t s = __byte_perm((uint32_t)tab[gp[m] & 0xFFFFu], (uint32_t)tab[gp[m] >> 16],
+                                       0x5410);
         h[m] = mul_bf16x2(s, up[m]);
     }
     return make_uint4(h[0], h[1], h[2], h[3]);
-}
-
-// out of line: only warps that meet a gate outside the table's range call it
-__device__ __noinline__ uint4 silu_mul8_any(uint4 g, uint4 u, const uint16_t *tab)
-{
-    uint32_t unused = 0;
-    return silu_mul8<true>(g, u, tab, unused);
 }
 
 // Filled row number v -> buffer row: expert p is the last one with cum[p] <=
@@ -171,13 +129,8 @@ template <bool FP8>
 EP_DEV void process_chunk(const Chunk &ch, const uint16_t *tab, int I, void *act,
                           float *act_scale)
 {
-    uint32_t bad = 0;
-    uint4 h0 = silu_mul8<false>(ch.g0, ch.u0, tab, bad);
-    uint4 h1 = silu_mul8<false>(ch.g1, ch.u1, tab, bad);
-    if (__any_sync(FULL_MASK, bad != 0)) {  // rare: a gate below 2^-25 or above 2^7
-        h0 = silu_mul8_any(ch.g0, ch.u0, tab);
-        h1 = silu_mul8_any(ch.g1, ch.u1, tab);
-    }
+    const uint4 h0 = silu_mul8(ch.g0, ch.u0, tab);
+    const uint4 h1 = silu_mul8(ch.g1, ch.u1, tab);
     if (FP8) {
         float scale;
         const uint4 q = quant::quant_chunk(h0, h1, scale);
@@ -198,11 +151,11 @@ silu_mul_kernel(const uint16_t *__restrict__ gate_up, int n_rows, int I,
                 const int32_t *__restrict__ expert_off, const int32_t *__restrict__ cnt_expert,
                 int P, void *__restrict__ act, float *__restrict__ act_scale)
 {
-    extern __shared__ int sm[];
-    int *cum = sm;            // [P + 1]  prefix sum of the counts
-    int *eoff = sm + P + 1;   // [P]      first buffer row of each expert
+    extern __shared__ __align__(16) int sm[];
+    uint16_t *tab = reinterpret_cast<uint16_t *>(sm);  // [TAB_SIZE] the SiLU table
+    int *cum = sm + TAB_SIZE / 2;  // [P + 1]  prefix sum of the counts
+    int *eoff = cum + P + 1;       // [P]      first buffer row of each expert
     __shared__ int warp_tot[ACT_THREADS / 32 + 1];
-    __shared__ __align__(16) uint16_t tab[TAB_SIZE];
     pdl_launch_dependents();
     // the table is no input of this call: copy it while the previous kernel
     // finishes
@@ -268,12 +221,21 @@ silu_mul_kernel(const uint16_t *__restrict__ gate_up, int n_rows, int I,
     }
 }
 
-size_t act_smem_bytes(int P) { return sizeof(int) * (size_t)(2 * P + 1); }
+size_t act_smem_bytes(int P)
+{
+    return sizeof(uint16_t) * TAB_SIZE + sizeof(int) * (size_t)(2 * P + 1);
+}
 
 }  // namespace
 
+// Called once per device before the first launch there: opts both instances
+// in to the shared memory of the largest expert count (128 KB of table plus
+// 32 KB of prefix sums at MAX_PHYS experts).
 int activation_blocks_per_sm()
 {
+    const int most = (int)act_smem_bytes(MAX_PHYS);
+    cudaFuncSetAttribute(silu_mul_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    cudaFuncSetAttribute(silu_mul_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, silu_mul_kernel<true>, ACT_THREADS,
                                                   act_smem_bytes(256));
@@ -285,11 +247,6 @@ cudaError_t launch_activation(const ActivationArgs &a, cudaStream_t s)
     if (a.n_rows == 0) return cudaSuccess;
     const int P = a.expert_off != nullptr ? a.P : 0;
     const size_t smem = act_smem_bytes(P);
-    const void *fn = a.fp8 ? (const void *)silu_mul_kernel<true> : (const void *)silu_mul_kernel<false>;
-    // the kernel also holds 16 KB of static shared memory (the SiLU table):
-    // opt in above the default 48 KB for the sum of the two
-    if (smem + sizeof(uint16_t) * TAB_SIZE + 1024 > 48 * 1024)
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     // without counts the work is known on the host: no more blocks than chunks
     long long blocks = a.grid;
     if (a.expert_off == nullptr) {

@@ -1,16 +1,20 @@
 /*
  * Build-time generator of the SiLU table used by the expert activation
- * kernel (activation.cu): for every bf16 gate g with 2^-25 <= |g| < 2^7, the
- * bf16 pattern of silu(g) = g / (1 + e^-g), correctly rounded to nearest
- * (ties to even).
+ * kernel (activation.cu): for every one of the 65,536 bf16 gate patterns g,
+ * the bf16 pattern of silu(g) = g / (1 + e^-g), correctly rounded to nearest
+ * (ties to even).  Entry i is the result for the gate whose bit pattern is i.
  *
- * Entry i = (sign << 12) | (|g| pattern - 0x3300), i.e. 8192 entries: the
- * magnitude patterns 0x3300 (2^-25) .. 0x42FF (just below 2^7) for each sign.
- *
- * Evaluated in x87 extended precision (64-bit significand): the relative
- * error of the quotient is a few units of 2^-64, and the generator stops with
- * an error if any value lies within 2^-56 (relative) of a bf16 rounding
- * midpoint, where that error could decide the rounding.  None does.
+ * For 2^-25 <= |g| < 2^7 the value is evaluated in x87 extended precision
+ * (64-bit significand): the relative error of the quotient is a few units of
+ * 2^-64, and the generator stops with an error if any value lies within
+ * 2^-56 (relative) of a bf16 rounding midpoint, where that error could decide
+ * the rounding.  None does.  Outside that range the result has closed forms:
+ *   |g| < 2^-25: silu(g) - g/2 = g tanh(g/2) / 2 is positive (g and
+ *     tanh(g/2) share a sign) and below half a bf16 step of g/2, so the
+ *     result is g/2 (exact in fp32) rounded to bf16 with ties toward +inf (a
+ *     tie occurs only below 2^-126);
+ *   |g| >= 2^7 and +-inf: g for g > 0 and -0 for g < 0 (|g e^g| < 2^-180);
+ *   NaN: the gate pattern itself.
  *
  * Usage: gen_silu_table > silu_table.inc  (comma-separated hex values)
  */
@@ -50,18 +54,38 @@ static uint16_t round_to_bf16(long double v, int *close)
     return (uint16_t)(sign | (u >> 16));
 }
 
+/* g/2 rounded to bf16, ties toward +inf: the low 16 bits of the fp32
+ * pattern decide, a tie (exactly 0x8000) going up in magnitude for g > 0 and
+ * down in magnitude for g < 0. */
+static uint16_t half_toward_plus_inf(uint16_t b)
+{
+    float h = bf16_to_float(b) * 0.5f;
+    uint32_t u;
+    memcpy(&u, &h, sizeof u);
+    return (uint16_t)((u + ((u >> 31) ? 0x7FFFu : 0x8000u)) >> 16);
+}
+
 int main(void)
 {
     int bad = 0;
-    for (int i = 0; i < 8192; ++i) {
-        uint16_t b = (uint16_t)(((i >> 12) << 15) | (0x3300 + (i & 4095)));
-        long double x = (long double)bf16_to_float(b);
-        long double v = x / (1.0L + expl(-x));
-        int close = 0;
-        uint16_t s = round_to_bf16(v, &close);
-        if (close) {
-            fprintf(stderr, "gen_silu_table: input 0x%04x lies too close to a midpoint\n", b);
-            bad = 1;
+    for (int i = 0; i < 65536; ++i) {
+        const uint16_t b = (uint16_t)i, a = b & 0x7FFFu;
+        uint16_t s;
+        if (a > 0x7F80u) {
+            s = b;
+        } else if (a >= 0x4300u) {
+            s = (b & 0x8000u) ? 0x8000u : b;
+        } else if (a < 0x3300u) {
+            s = half_toward_plus_inf(b);
+        } else {
+            long double x = (long double)bf16_to_float(b);
+            long double v = x / (1.0L + expl(-x));
+            int close = 0;
+            s = round_to_bf16(v, &close);
+            if (close) {
+                fprintf(stderr, "gen_silu_table: input 0x%04x lies too close to a midpoint\n", b);
+                bad = 1;
+            }
         }
         printf("0x%04x,%s", s, (i % 16 == 15) ? "\n" : " ");
     }
