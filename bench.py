@@ -268,9 +268,9 @@ def main():
     ap.add_argument("--config", default="v3", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--schedule", default="micro", choices=["micro", "sequential"],
-                    help="micro: two micro-batches in flight (route+layout of batch i+1 "
-                         "overlap dispatch+combine of batch i); sequential: one step after "
-                         "the other on one stream")
+                    help="micro: micro-batches in flight over three buffer sets (route+layout "
+                         "of later batches overlap dispatch+combine of batch i); sequential: "
+                         "one step after the other on one stream")
     ap.add_argument("--num-sms", type=int, default=0)
     ap.add_argument("--split-sms", default="",
                     help="micro-batch schedule: 'd,c' runs dispatch of batch i+1 on d SMs next "
@@ -428,7 +428,7 @@ def main():
     seq_ms = graph_ms
     value_seq = tokens_per_s(cfg.T, world, K, seq_ms)
 
-    # 3. the same K batches with two micro-batches in flight
+    # 3. the same K batches with micro-batches in flight (three buffer sets)
     micro_ms = None
     # the two-stream schedule has no L2 flush between steps, so it is only
     # timed when a step's data is larger than L2 anyway
@@ -730,9 +730,10 @@ def main():
                               if flush else
                               f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB moved per step)"),
                        "parallelism": f"replicas x{world}",
-                       "schedule": ("two micro-batches in flight: route+layout of batch i+1 "
-                                    "on one stream overlap dispatch+combine of batch i on "
-                                    "another" if micro_ms is not None else
+                       "schedule": ("micro-batches in flight over three buffer sets: "
+                                    "route+layout of later batches on one stream overlap "
+                                    "dispatch+combine of batch i on another"
+                                    if micro_ms is not None else
                                     "sequential, one stream, step replayed as a CUDA graph")},
             "value_sequential": value_seq, "ms_per_step_sequential": seq_ms / K,
             "value_sequential_eager": tokens_per_s(cfg.T, world, K, eager_ms),

@@ -233,23 +233,29 @@ class EpHostPipeline:
 
 
 class EpMicroBatchPipeline:
-    """Two micro-batches in flight, as in the two-micro-batch overlap of
+    """Micro-batches in flight, as in the two-micro-batch overlap of
     DeepSeek's and Perplexity's EP deployments.
 
     Routing and layout (arithmetic- and latency-bound) run on one stream.
     With ``split_sms=None`` dispatch and combine of a batch follow each other
-    on a second stream, overlapping the next batch's routing.  With
+    on a second stream, overlapping later batches' routing.  With
     ``split_sms=(d, c)`` they get a stream each and are capped to d and c SMs,
     so the write-heavy dispatch of batch i+1 runs next to the read-heavy
     combine of batch i and HBM sees a mix of reads and writes instead of a
-    pure write phase followed by a pure read phase.  Each of the two
-    ``EpPath`` buffer sets serves every other batch; batch i+2 starts its
-    routing only after batch i has finished its combine.
+    pure write phase followed by a pure read phase.  Batch i uses buffer set
+    i mod ``n_sets`` (one ``EpPath`` each) and starts its routing only after
+    batch i - n_sets has finished its combine.  With three sets the routing
+    of a batch is released together with the dispatch two batches earlier,
+    every time, so the two share the GPU the same way in every step (with two
+    sets the routing's start drifts against the dispatch and the step time
+    moves between two levels).
     """
 
-    def __init__(self, make_path, device="cuda", split_sms=None):
+    def __init__(self, make_path, device="cuda", split_sms=None, n_sets: int = 3):
+        if n_sets < 2:
+            raise ValueError("n_sets must be at least 2")
         dev = torch.device(device)
-        self.paths = [make_path(), make_path()]
+        self.paths = [make_path() for _ in range(n_sets)]
         self.split = split_sms
         if split_sms is not None:
             for p in self.paths:
@@ -257,7 +263,7 @@ class EpMicroBatchPipeline:
         self.s_route = torch.cuda.Stream(dev)
         self.s_move = torch.cuda.Stream(dev)     # dispatch (and combine unless split)
         self.s_comb = torch.cuda.Stream(dev) if split_sms is not None else self.s_move
-        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        ev = lambda: [torch.cuda.Event() for _ in range(n_sets)]  # noqa: E731
         self.layout_done, self.disp_done, self.move_done = ev(), ev(), ev()
 
     @property
@@ -267,12 +273,13 @@ class EpMicroBatchPipeline:
 
     def run(self, xs, logits, biases, ys):
         """Enqueues batch i = (xs[i], logits[i], biases[i], expert outputs
-        ys[i]); results land in ``self.paths[i % 2].out``.  Returns without
-        synchronising; ``self.s_last`` carries the last combine."""
+        ys[i]); results land in ``self.paths[i % n_sets].out``.  Returns
+        without synchronising; ``self.s_last`` carries the last combine."""
+        n = len(self.paths)
         for i in range(len(xs)):
-            b = i & 1
+            b = i % n
             p = self.paths[b]
-            if i >= 2:  # buffer set b is free once batch i-2 has combined
+            if i >= n:  # buffer set b is free once batch i-n has combined
                 self.s_route.wait_event(self.move_done[b])
             with torch.cuda.stream(self.s_route):
                 p.route_layout(logits[i], biases[i], stream=self.s_route)
