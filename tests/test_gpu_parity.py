@@ -223,6 +223,41 @@ def test_layout_empty():
         assert (getattr(path, n) == 0).all(), n
 
 
+def test_empty_batch_every_call():
+    """T = 0 through every call that moves rows: each returns without
+    touching its outputs, and the fused decode call writes the empty layout
+    (zero counts and offsets) like ep_route_layout"""
+    from combine_ep_route_02_b200 import (ep_combine, ep_combine_backward, ep_dispatch,
+                                          ep_dispatch_backward)
+    H, k = 7168, 8
+    x = torch.empty((0, H), dtype=torch.bfloat16, device="cuda")
+    slot = torch.empty((0, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((0, k), dtype=torch.float32, device="cuda")
+    recv_x = torch.full((4, H), 0x5A, dtype=torch.uint8, device="cuda")
+    recv_s = torch.full((4, H // 128), 3.0, dtype=torch.float32, device="cuda")
+    y = torch.ones((4, H), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((1, H), 5.0, dtype=torch.bfloat16, device="cuda")
+    gw = torch.full((1, k), 7.0, dtype=torch.float32, device="cuda")
+    st = torch.full((1,), 9, dtype=torch.int32, device="cuda")
+    ep_dispatch(x, 0, H, k, slot, True, recv_x, recv_s, dev_status=st, recv_rows=4)
+    ep_combine(y, slot, w, 0, H, k, out, recv_rows=4)
+    ep_dispatch_backward(y, slot, 0, H, k, out, recv_rows=4)
+    ep_combine_backward(x, y, slot, w, 0, H, k, y, gw, recv_rows=4)
+    torch.cuda.synchronize()
+    assert (recv_x == 0x5A).all() and (recv_s == 3.0).all()
+    assert (out == 5.0).all() and (y == 1.0).all() and (gw == 7.0).all()
+    cfg = CONFIGS["v3_decode"].scaled(0)
+    wl = Workload(cfg)
+    path = make_path(cfg, wl)
+    for n in ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank"):
+        getattr(path, n).fill_(-5)
+    path.route_dispatch(wl.logits.cuda(), wl.bias.cuda(), wl.x.cuda())
+    torch.cuda.synchronize()
+    path.check_status()
+    for n in ("cnt_expert", "expert_off", "rows_rank", "rank_off", "tok_rank"):
+        assert (getattr(path, n) == 0).all(), n
+
+
 @pytest.mark.parametrize("T", [700, 20000])
 def test_layout_max_sizes_and_skewed_ids(T):
     """P = 4096 physical experts, k = 32, R = 64, heavily skewed expert ids;
