@@ -167,26 +167,6 @@ EP_DEV void sts128(uint32_t addr, uint4 v)
 EP_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 EP_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// (value desc, index asc) total order used by every selection.
-EP_DEV bool beats(float va, int ia, float vb, int ib)
-{
-    return va > vb || (va == vb && ia < ib);
-}
-
-// Butterfly arg-max over the warp; every lane ends with the winner.
-EP_DEV void warp_argmax(float &v, int &i)
-{
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        float ov = __shfl_xor_sync(FULL_MASK, v, off);
-        int oi = __shfl_xor_sync(FULL_MASK, i, off);
-        if (beats(ov, oi, v, i)) {
-            v = ov;
-            i = oi;
-        }
-    }
-}
-
 EP_DEV int warp_inclusive_scan(int v)
 {
     const int lane = threadIdx.x & 31;

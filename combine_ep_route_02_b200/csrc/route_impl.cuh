@@ -5,12 +5,15 @@
 // section) with plain top-k as its one-group special case (Perplexity blog,
 // section "MoE Router").  Lane l holds experts [l*EPL, (l+1)*EPL).
 //
-// Every arg-max (groups, then each of the k experts) is two warp reductions
-// on integers: redux.sync max over an order-preserving 32-bit image of the
-// fp32 key, then redux.sync min over the indices of the lanes holding that
-// maximum, which is exactly the (key desc, index asc) order.  Keys are never
-// -0.0 or NaN here (s >= 0, and s + b rounds an exact zero to +0), so the
-// integer order equals the fp32 order.
+// Keys are compared as an order-preserving 32-bit image of the fp32 key.
+// Keys are never -0.0 or NaN here (s >= 0, and s + b rounds an exact zero to
+// +0), so the integer order equals the fp32 order.  The kept groups are the
+// first topk_group in (score desc, id asc) order, found by ranking every
+// group against all the others.  Each of the k experts is then one warp
+// reduction: redux.sync max over the lanes' best keys, and the lowest lane
+// holding that maximum (a ballot) owns the pick: lanes hold ascending index
+// ranges and each lane's best is the lowest index of its largest key, so
+// this is exactly the (key desc, index asc) order.
 //
 // When a group is a power-of-two number of whole lanes (E/G a multiple of
 // EPL), each lane sits in one group and the group top-2 is a butterfly over
@@ -216,14 +219,6 @@ static __device__ __noinline__ float sigmoid_exact(float x)
     return (__float_as_uint(lo32) & 1u) ? hi32 : lo32;  // a tie: to even (never met)
 }
 
-// winner of (key desc, index asc) over the warp; every lane gets it
-EP_DEV int warp_pick(uint32_t key, int idx)
-{
-    const uint32_t kmax = __reduce_max_sync(FULL_MASK, key);
-    const uint32_t cand = (key == kmax) ? (uint32_t)idx : 0xffffffffu;
-    return (int)__reduce_min_sync(FULL_MASK, cand);
-}
-
 // Bias and token-invariant group id of each expert a lane holds (lane l
 // holds experts [l*EPL, (l+1)*EPL)); -1: no such expert.
 template <int EPL>
@@ -270,8 +265,11 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
     }
 
     if (G > 1) {
-        // group score = fp32 sum of the two largest keys in the group
-        uint32_t chosen = 0;
+        // group score = fp32 sum of the two largest keys in the group; the
+        // lane that holds group g's score (every lane of the group when
+        // aligned, lane g otherwise)
+        uint32_t my_score = NONE;
+        int score_lane_step = 1;
         if (aligned) {
             float a1 = -INFINITY, a2 = -INFINITY;
 #pragma unroll
@@ -294,15 +292,9 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
                 a1 = fmaxf(a1, o1);
                 a2 = n2;
             }
-            const uint32_t my_score =
-                (my_group >= 0) ? ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f)) : NONE;
-            for (int r = 0; r < Kg; ++r) {
-                const bool cand = my_group >= 0 && !((chosen >> my_group) & 1u);
-                const int g = warp_pick(cand ? my_score : NONE, cand ? my_group : 0x7fffffff);
-                chosen |= 1u << g;
-            }
+            if (my_group >= 0) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
+            score_lane_step = lanes_per_group;
         } else {
-            uint32_t my_score = NONE;  // lane g keeps the score of group g
             for (int g = 0; g < G; ++g) {
                 float a1 = -INFINITY, a2 = -INFINITY;
 #pragma unroll
@@ -326,12 +318,19 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
                 }
                 if (lane == g) my_score = ordered(__fadd_rn(__fadd_rn(a1, a2), 0.0f));
             }
-            for (int r = 0; r < Kg; ++r) {
-                const bool cand = lane < G && !((chosen >> lane) & 1u);
-                const int g = warp_pick(cand ? my_score : NONE, cand ? lane : 0x7fffffff);
-                chosen |= 1u << g;
-            }
         }
+        // the Kg groups first in (score descending, id ascending) order:
+        // lane g < G ranks group g against every group and keeps it when
+        // fewer than Kg come before it (the same set as Kg successive
+        // arg-max picks with ties to the lower id)
+        const int gl = lane < G ? lane : 0;
+        const uint32_t sc_mine = __shfl_sync(FULL_MASK, my_score, gl * score_lane_step);
+        int before = 0;
+        for (int g = 0; g < G; ++g) {
+            const uint32_t sc = __shfl_sync(FULL_MASK, my_score, g * score_lane_step);
+            before += (sc > sc_mine || (sc == sc_mine && g < gl)) ? 1 : 0;
+        }
+        const uint32_t chosen = __ballot_sync(FULL_MASK, lane < G && before < Kg);
         if (aligned) {
             // the lane's experts share one group
             if (my_group >= 0 && !((chosen >> my_group) & 1u))
@@ -358,25 +357,30 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
     int sel_idx = 0;
     float sel_s = 0.0f;
     for (int r = 0; r < k; ++r) {
-        const int e = warp_pick(best_k, best_i);
-        const int owner = e / EPL;  // k <= eligible experts, so e is real
+        // the largest key; among equal ones the lowest lane holds the lowest
+        // index (lanes own ascending index ranges), and its best_i is the
+        // lowest index of that key in the lane
+        const uint32_t kmax = __reduce_max_sync(FULL_MASK, best_k);
+        const int owner = __ffs(__ballot_sync(FULL_MASK, best_k == kmax)) - 1;
+        const int e = __shfl_sync(FULL_MASK, best_i, owner);
+        // every lane runs the owner's update; only the owner keeps it (no
+        // divergent branch inside the pick loop)
+        const bool own = lane == owner;
+        const int mine = best_i;
         float sv = 0.0f;
-        if (lane == owner) {
+        uint32_t nk = NONE;
+        int ni = 0x7fffffff;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (e0 + i == e) {
-                    sv = s[i];
-                    key[i] = NONE;
-                }
-            best_k = NONE;
-            best_i = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (key[i] > best_k) {
-                    best_k = key[i];
-                    best_i = e0 + i;
-                }
+        for (int i = 0; i < EPL; ++i) {
+            const bool hit = own && (e0 + i == mine);
+            sv = hit ? s[i] : sv;
+            key[i] = hit ? NONE : key[i];
+            const bool better = key[i] > nk;
+            nk = better ? key[i] : nk;
+            ni = better ? e0 + i : ni;
         }
+        best_k = own ? nk : best_k;
+        best_i = own ? ni : best_i;
         sv = __shfl_sync(FULL_MASK, sv, owner);
         if (lane == r) {
             sel_idx = e;
