@@ -219,6 +219,32 @@ static __device__ __noinline__ float sigmoid_exact(float x)
     return (__float_as_uint(lo32) & 1u) ? hi32 : lo32;  // a tie: to even (never met)
 }
 
+// The lane's best key and its expert: the first (lowest index) of the
+// largest keys, by a tree of pairwise picks (the right half of a pair wins
+// only with a strictly larger key), so the dependency chain is log2(EPL)
+// steps long.  EPL is a power of two.
+template <int EPL>
+EP_DEV void lane_best(const uint32_t (&key)[EPL], int e0, uint32_t &best_k, int &best_i)
+{
+    uint32_t tk[EPL];
+    int ti[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        tk[i] = key[i];
+        ti[i] = e0 + i;
+    }
+#pragma unroll
+    for (int w = EPL / 2; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) {
+            const bool right = tk[2 * j + 1] > tk[2 * j];
+            tk[j] = right ? tk[2 * j + 1] : tk[2 * j];
+            ti[j] = right ? ti[2 * j + 1] : ti[2 * j];
+        }
+    best_k = tk[0];
+    best_i = ti[0];
+}
+
 // Bias and token-invariant group id of each expert a lane holds (lane l
 // holds experts [l*EPL, (l+1)*EPL)); -1: no such expert.
 template <int EPL>
@@ -344,15 +370,11 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
     }
 
     // lane-local best: the first (lowest index) of the largest keys;
-    // excluded and taken experts hold NONE, below every real key
-    uint32_t best_k = NONE;
-    int best_i = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i)
-        if (key[i] > best_k) {
-            best_k = key[i];
-            best_i = e0 + i;
-        }
+    // excluded and taken experts hold NONE, below every real key (a lane
+    // whose keys are all NONE is never the owner of a pick)
+    uint32_t best_k;
+    int best_i;
+    lane_best<EPL>(key, e0, best_k, best_i);
 
     int sel_idx = 0;
     float sel_s = 0.0f;
@@ -368,17 +390,15 @@ EP_DEV void select_topk(float (&s)[EPL], const float (&b)[EPL], const int (&gid)
         const bool own = lane == owner;
         const int mine = best_i;
         float sv = 0.0f;
-        uint32_t nk = NONE;
-        int ni = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             const bool hit = own && (e0 + i == mine);
             sv = hit ? s[i] : sv;
             key[i] = hit ? NONE : key[i];
-            const bool better = key[i] > nk;
-            nk = better ? key[i] : nk;
-            ni = better ? e0 + i : ni;
         }
+        uint32_t nk;
+        int ni;
+        lane_best<EPL>(key, e0, nk, ni);
         best_k = own ? nk : best_k;
         best_i = own ? ni : best_i;
         sv = __shfl_sync(FULL_MASK, sv, owner);
