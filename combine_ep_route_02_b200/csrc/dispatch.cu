@@ -91,11 +91,16 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
 //     shared memory, each completing on its own mbarrier;
 //   - all threads quantise the row from shared memory into an output stage
 //     (H code bytes + H/128 fp32 scales);
-//   - lanes j < k of warp 0 each send the stage to receive row slot[t, j]
-//     with two bulk stores and track them in their own bulk groups, so an
-//     output stage is reused only after its previous stores have read it.
+//   - lanes j < k of warp 0 each send the stage's codes to receive row
+//     slot[t, j] with one bulk store and track it in their own bulk group,
+//     so an output stage is reused only after its previous stores have read
+//     it; meanwhile warps 1.. copy the stage's scale row (H/128 floats) to
+//     the k scale rows with ordinary coalesced stores.
 // Memory traffic is issued by the TMA engine, so the threads' own loads and
-// stores no longer bound the number of bytes in flight.
+// stores no longer bound the number of bytes in flight.  The engine takes
+// its copies one after another at a cost per copy that hardly depends on
+// the size, so the small scale rows go by thread stores and each token
+// costs k copies, not 2k.
 // ---------------------------------------------------------------------------
 constexpr int TMA_IN_STAGES = 4;
 constexpr int TMA_OUT_STAGES = 4;
@@ -123,6 +128,7 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int first = blockIdx.x, step = gridDim.x;
     const int n_my = (first < T) ? (T - first + step - 1) / step : 0;
+    __shared__ int slot_sh[32];  // this token's k receive rows (k <= 32)
 
     pdl_launch_dependents();
     if (tid == 0) {
@@ -146,7 +152,10 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
         const int st = it % TMA_IN_STAGES;
         const int o = it % TMA_OUT_STAGES;
         int my_slot = -1;
-        if (warp == 0 && lane < k) my_slot = __ldg(slot + (size_t)t * k + lane);
+        if (warp == 0 && lane < k) {
+            my_slot = __ldg(slot + (size_t)t * k + lane);
+            slot_sh[lane] = my_slot;  // read by the scale-row warps below
+        }
         const bool ok = mbar_wait(bar_base + 8 * st, (it / TMA_IN_STAGES) & 1, wait_limit);
         if (!__syncthreads_and(ok)) {
             failed_at = it;
@@ -183,14 +192,25 @@ dispatch_fp8_tma_kernel(const uint16_t *__restrict__ x, int T, int H, int k,
                 bulk_load(in, x + (size_t)t2 * H, in_bytes, bar_base + 8 * st);
             }
             if (lane < k) {
-                if ((unsigned)my_slot < (unsigned)n_rows) {
+                if ((unsigned)my_slot < (unsigned)n_rows)
                     bulk_store(recv_x + (size_t)my_slot * H, qo, (uint32_t)H);
-                    bulk_store(recv_scale + (size_t)my_slot * S, so, (uint32_t)S * 4u);
-                }
                 bulk_commit();
                 // the stage written next iteration was sent TMA_OUT_STAGES-1
                 // groups ago: wait until those stores have read it
                 bulk_wait_read<TMA_OUT_STAGES - 1>();
+            }
+        } else {
+            // scale row j by warp 1 + (j mod (warps - 1)), lanes over its
+            // H/128 floats
+            const int nw = (int)(blockDim.x >> 5) - 1;
+            for (int j = warp - 1; j < k; j += nw) {
+                const int sj = slot_sh[j];
+                if ((unsigned)sj < (unsigned)n_rows)
+                    for (int c = lane; c < S; c += 32) {
+                        float v;
+                        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(so + 4u * c));
+                        st_stream_f32(recv_scale + (size_t)sj * S + c, v);
+                    }
             }
         }
         __syncthreads();
