@@ -29,7 +29,8 @@ namespace {
 
 using namespace layout_impl;
 
-__global__ void __launch_bounds__(LAYOUT_THREADS) layout_count_kernel(LayoutArgs a)
+template <int NTH>
+__global__ void __launch_bounds__(NTH) layout_count_kernel(LayoutArgs a)
 {
     extern __shared__ int smem[];
     __shared__ int bad_sh;
@@ -70,14 +71,14 @@ __global__ void __launch_bounds__(SCAN_THREADS) layout_scan_kernel(LayoutArgs a)
     }
 }
 
-template <bool FUSED>
-__global__ void __launch_bounds__(LAYOUT_THREADS) layout_slot_kernel(LayoutArgs a)
+template <int NTH, bool FUSED>
+__global__ void __launch_bounds__(NTH) layout_slot_kernel(LayoutArgs a)
 {
     extern __shared__ int smem[];
-    __shared__ int warp_tot[LAYOUT_WARPS + 1];
+    __shared__ int warp_tot[NTH / 32 + 1];
     pdl_launch_dependents();
     pdl_wait();
-    slot_tile<LAYOUT_THREADS, FUSED>(a, blockIdx.x, smem, warp_tot);
+    slot_tile<NTH, FUSED>(a, blockIdx.x, smem, warp_tot);
 }
 
 __global__ void layout_empty_kernel(LayoutArgs a)
@@ -102,29 +103,47 @@ void opt_in_smem(const void *fn, size_t bytes)
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-}  // namespace
-
-cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
+// The count and slot kernels for blocks of NTH threads.
+template <int NTH>
+cudaError_t launch_tiles(const LayoutArgs &a, cudaStream_t s)
 {
     cudaError_t err;
-    if (a.T == 0) return launch_pdl(layout_empty_kernel, dim3(1), dim3(256), 0, s, a);
     const int NT = a.n_tiles;
     const size_t pairs = (size_t)a.tile_tokens * a.k;
     const size_t sm_count = sizeof(int) * count_smem_ints(a.P, a.R, a.tile_tokens, a.k);
     const size_t sm_slot =
         sizeof(int) * ((size_t)2 * a.P + 1 + (size_t)a.hist_warps * a.P + pairs);
     const bool fused = NT <= LAYOUT_FUSED_MAX_TILES;
-    opt_in_smem((const void *)layout_count_kernel, sm_count);
-    opt_in_smem(fused ? (const void *)layout_slot_kernel<true> : (const void *)layout_slot_kernel<false>,
+    opt_in_smem((const void *)layout_count_kernel<NTH>, sm_count);
+    opt_in_smem(fused ? (const void *)layout_slot_kernel<NTH, true>
+                      : (const void *)layout_slot_kernel<NTH, false>,
                 sm_slot);
-    err = launch_pdl(layout_count_kernel, dim3(NT), dim3(LAYOUT_THREADS), sm_count, s, a);
+    err = launch_pdl(layout_count_kernel<NTH>, dim3(NT), dim3(NTH), sm_count, s, a);
     if (err != cudaSuccess) return err;
-    if (fused) return launch_pdl(layout_slot_kernel<true>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
+    if (fused)
+        return launch_pdl(layout_slot_kernel<NTH, true>, dim3(NT), dim3(NTH), sm_slot, s, a);
     const int cols = a.P + a.R;
     err = launch_pdl(layout_scan_kernel, dim3((cols + SCAN_WARPS - 1) / SCAN_WARPS),
                      dim3(SCAN_THREADS), 0, s, a);
     if (err != cudaSuccess) return err;
-    return launch_pdl(layout_slot_kernel<false>, dim3(NT), dim3(LAYOUT_THREADS), sm_slot, s, a);
+    return launch_pdl(layout_slot_kernel<NTH, false>, dim3(NT), dim3(NTH), sm_slot, s, a);
+}
+
+}  // namespace
+
+cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s)
+{
+    if (a.T == 0) return launch_pdl(layout_empty_kernel, dim3(1), dim3(256), 0, s, a);
+    // Tiles of at most 512 pairs take blocks of 512 threads: every phase of
+    // the two kernels ends in a block barrier, and with a small tile most of
+    // 32 warps would only wait at them.  The slot kernel's ordering warps
+    // (hist_warps) cannot outnumber the block's warps.
+    if ((long long)a.tile_tokens * a.k <= 512) {
+        LayoutArgs b = a;
+        if (b.hist_warps > 512 / 32) b.hist_warps = 512 / 32;
+        return launch_tiles<512>(b, s);
+    }
+    return launch_tiles<LAYOUT_THREADS>(a, s);
 }
 
 }  // namespace ep
