@@ -121,7 +121,6 @@ route_dispatch_small_kernel(RouteArgs r, LayoutArgs a, DecodeArgs d, int vec4)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ double tab[64];
-    __shared__ int warp_tot[DEC_WARPS + 1];
     __shared__ int bad_sh, xfail_sh, go_sh;
     __shared__ __align__(8) uint64_t xbar;
 
@@ -234,12 +233,26 @@ route_dispatch_small_kernel(RouteArgs r, LayoutArgs a, DecodeArgs d, int vec4)
         __syncthreads();
         status |= bad_sh;  // every block finds the same bits
         const int A = a.row_align;
-        for (int p = tid; p < P; p += DEC_THREADS) eoff[p] = (hist[p] + A - 1) / A * A;
+        if (warp == 0) {
+            // exclusive scan of the padded counts by one warp (one block
+            // barrier instead of several): lane l takes experts
+            // [l * per, (l + 1) * per), per <= 32 since P <= 1024
+            const int per = (P + 31) >> 5;
+            const int lo = min(P, lane * per), hi = min(P, lo + per);
+            int local = 0;
+            for (int p = lo; p < hi; ++p) local += (hist[p] + A - 1) / A * A;
+            const int incl = warp_inclusive_scan(local);
+            int acc = incl - local;
+            for (int p = lo; p < hi; ++p) {
+                const int c = (hist[p] + A - 1) / A * A;
+                eoff[p] = acc;
+                run[p] += acc;  // the block's first row of expert p
+                acc += c;
+            }
+            if (lane == 31) eoff[P] = incl;
+        }
         __syncthreads();
-        const int total = layout_impl::block_exclusive_scan<DEC_THREADS>(eoff, P, warp_tot);
-        if (tid == 0) eoff[P] = total;
-        for (int p = tid; p < P; p += DEC_THREADS) run[p] += eoff[p];
-        __syncthreads();
+        const int total = eoff[P];
 
         const int epr = P / R;  // rank q holds experts [q * epr, (q + 1) * epr)
         if (warp == 0) {
