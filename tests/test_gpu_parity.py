@@ -199,9 +199,12 @@ def test_layout_full_size(name):
         assert np.array_equal(got[n].reshape(ref[n].shape), ref[n]), n
 
 
-@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 1000, 4097, 40000])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 1000, 4096, 4097, 5440, 5441, 40000])
 @pytest.mark.parametrize("name", ["ds16b", "skew"])
 def test_layout_ragged(T, name):
+    """ragged batches, and both sides of the block-size switch (tiles of at
+    most 512 pairs run 512-thread blocks: top-8 up to T = 4096, top-6 up to
+    T = 5440)"""
     cfg = CONFIGS[name].scaled(T)
     wl = Workload(cfg, seed=T)
     idx, _, _ = oracle_route(cfg, wl)
