@@ -420,6 +420,32 @@ def test_dispatch_num_sms_and_invalid_slots(num_sms):
     assert (got[unwritten] == 0xAB).all() and (gs[unwritten] == -1.0).all()
 
 
+@pytest.mark.parametrize("k", [1, 13, 14, 32])
+def test_dispatch_tma_topk(k):
+    """the TMA pipeline at H = 7168 (14 warps: warp 0 issues the code rows'
+    bulk copies, the other 13 write the k scale rows, several each from
+    k = 14) with invalid slots, against the oracle"""
+    from combine_ep_route_02_b200 import ep_dispatch
+    T, H = 97, 7168
+    g = torch.Generator().manual_seed(k)
+    x = (torch.randn((T, H), generator=g) * 3).to(torch.bfloat16)
+    rng = np.random.default_rng(k)
+    slot = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    slot[0, k - 1] = -1
+    slot[T - 1, 0] = T * k
+    rx = torch.full((T * k, H), 0x5A, dtype=torch.uint8, device="cuda")
+    rs = torch.full((T * k, H // 128), -2.0, dtype=torch.float32, device="cuda")
+    ep_dispatch(x.cuda(), T, H, k, torch.from_numpy(slot).cuda(), True, rx, rs)
+    torch.cuda.synchronize()
+    ref_x, ref_s = oracle.dispatch(x, slot, True)
+    ok = slot[(slot >= 0) & (slot < T * k)]
+    untouched = np.setdiff1d(np.arange(T * k), ok)
+    got_x, got_s = rx.cpu().numpy(), rs.cpu().numpy()
+    assert np.array_equal(got_x[ok], ref_x[ok])
+    assert np.array_equal(got_s[ok].view(np.uint32), ref_s[ok].view(np.uint32))
+    assert (got_x[untouched] == 0x5A).all() and (got_s[untouched] == -2.0).all()
+
+
 def test_dispatch_fp8_thread_store_path():
     """a recv_scale that is 4- but not 16-byte aligned takes the thread-store
     kernel instead of the TMA pipeline; both must give the oracle's bytes"""
